@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Benchmark of the expert-routed MoE FFN layer on B200.
+
+A step is one full layer call (route -> plan -> grouped gate/up + SwiGLU -> grouped
+down -> combine) over one batch of synthetic hidden states, on weights resident in
+HBM. Default workload: 1-token decode (d=2560, E=512, top-10 + 1 shared, f=1024,
+int4 g128). Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+
+L2: each step reads a different copy of the layer's weights (``replicas`` copies,
+cycled) and a different hidden batch (a pool of 64), so no step finds its weights in
+the 126 MB L2 (the inputs of the cycle are far larger than L2).
+Multi-GPU: every rank runs its own replica of the layer (weak scaling, no data-path
+collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from expert_routed_ffn_route_b200 import synth  # noqa: E402
+
+HBM_FALLBACK_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+POOL = 64
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=list(synth.CONFIGS))
+    ap.add_argument("--replicas", type=int, default=0, help="weight copies cycled (0: auto)")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return HBM_FALLBACK_GBS, "fallback"
+
+
+def bank_bytes_per_expert(cfg):
+    bits = synth.FMT_BITS[cfg.fmt]
+    w = 3 * cfg.d * cfg.f * bits // 8
+    s = 0 if cfg.fmt == "bf16" else 3 * cfg.d * cfg.f // cfg.group * 2
+    return w, s
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_rate(cfg, L, seconds):
+    """Tokens/s of the fp64 oracle on this host, on a bounded sample of the workload:
+    whole calls of up to 1 token each on successive tokens until `seconds` pass."""
+    from oracle import moe_oracle as O
+
+    def bank_dict(b):
+        if b is None:
+            return None
+        d = b.arrays()
+        d.update(fmt=b.fmt, group=b.group)
+        return d
+    routed, shared = bank_dict(L.routed), bank_dict(L.shared)
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        t = done % L.x.shape[0]
+        O.layer_forward(L.x[t:t + 1], L.router_w, L.router_bias, routed, shared, cfg.k)
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        pass
+    return done / el, cores, f"{done} single-token layer calls of '{cfg.name}' in {el:.1f} s"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def launches_per_step(T, k):
+    # router, top-k, plan (1 kernel up to 1024 assignments, else 3), gate/up, down, combine
+    return 2 + (1 if T * k <= 1024 else 3) + 3
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from expert_routed_ffn_route_b200 import binding as B
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synth.CONFIGS[args.workload]
+    B.load_library()
+
+    # ---- inputs
+    routed = synth.make_bank(cfg, "routed")
+    shared = synth.make_bank(cfg, "shared")
+    L = synth.make_layer(cfg, routed=routed, shared=shared)
+    pool = [L.x] + [synth.make_hidden(cfg, L.router_w, L.router_bias, stream=f"pool{i}")
+                    for i in range(1, POOL)]
+    base = B.DeviceLayer(L, device=dev)
+    x_dev = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in pool]
+
+    w_b, s_b = bank_bytes_per_expert(cfg)
+    per_exp = w_b + s_b
+    router_b = cfg.E * cfg.d * 2
+    # replicas: enough weight copies that a cycle touches > 4x L2
+    if args.replicas > 0:
+        R = args.replicas
+    else:
+        touched = min(cfg.E, cfg.T * cfg.k) + 1
+        step_bytes = touched * per_exp + router_b
+        R = int(min(16, max(1, np.ceil(4 * L2_BYTES / step_bytes))))
+    layers = [base]
+    for _ in range(R - 1):
+        b2 = {}
+        for name, bank in base.banks.items():
+            b2[name] = None if bank is None else {
+                k: (v.clone() if hasattr(v, "clone") else v) for k, v in bank.items()}
+        layers.append(B.DeviceLayer.from_tensors(
+            cfg, base.router_w.clone(),
+            None if base.router_bias is None else base.router_bias.clone(),
+            b2["routed"], b2["shared"]))
+    descs = [l.descriptor(cfg.T) for l in layers]
+    ws = B.alloc_workspace(descs[0], device=dev)
+    out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
+    idx_buf = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+
+    # ---- algorithmic bytes of the dominant kernel (grouped gate/up) per pool entry
+    gu_bytes, layer_bytes = [], []
+    for xd in x_dev:
+        B.layer_forward(descs[0], xd, ws, out=out, topk_idx=idx_buf)
+        u = np.unique(idx_buf.cpu().numpy()).size + (1 if L.shared is not None else 0)
+        gu = u * (2 * per_exp // 3) + cfg.T * cfg.d * 2 + (cfg.T * cfg.k + cfg.T) * cfg.f * 2
+        gu_bytes.append(gu)
+        layer_bytes.append(u * per_exp + router_b + 2 * cfg.T * cfg.d * 2)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+    n_cap = min(args.steps, R * 8)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n_cap)]
+    for a, b in ev:  # torch creates the CUDA event on its first record
+        a.record(stream)
+        b.record(stream)
+
+    def step(i, marks=None):
+        B.layer_forward(descs[i % R], x_dev[i % POOL], ws, out=out, marks=marks, stream=stream)
+
+    def marks_for(i):
+        m = [None] * B.N_MARKS
+        m[2], m[3] = ev[i % n_cap]
+        return m
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, marks_for(i))
+    torch.cuda.synchronize()
+
+    graphs = None
+    if not args.no_graph:
+        graphs = []
+        for i in range(n_cap):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(i, marks_for(i))
+            graphs.append(g)
+        with torch.cuda.stream(stream):
+            for g in graphs:
+                g.replay()
+        torch.cuda.synchronize()
+
+    # ---- timed region
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            for i in range(args.steps):
+                if graphs is not None:
+                    graphs[i % n_cap].replay()
+                else:
+                    step(i, marks_for(i))
+            t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+
+    # dominant kernel: the captured steps' gate/up launches (the last replay of each graph)
+    last = range(max(0, args.steps - n_cap), args.steps)
+    k_ms = [ev[i % n_cap][0].elapsed_time(ev[i % n_cap][1]) for i in last]
+    k_bytes = [gu_bytes[i % POOL] for i in last]
+    gu_avg_ms = float(np.mean(k_ms))
+    achieved = float(np.sum(k_bytes) / (np.sum(k_ms) * 1e-3) / 1e9)
+
+    # ---- end to end through the public call with host buffers
+    x_host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+              for x in pool[:8]]
+    out_host = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16).pin_memory()
+    x_stage = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
+    e_steps = min(args.steps, 200)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e_steps):
+            x_stage.copy_(x_host[i % len(x_host)], non_blocking=True)
+            B.layer_forward(descs[i % R], x_stage, ws, out=out, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    status = B.device_status(descs[0], ws)
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    peak, peak_kind = measured_peaks()
+    ms_per_step = ms / args.steps
+    res = {
+        "metric": f"MoE-layer tokens/s ({cfg.name}, T={cfg.T})",
+        "value": world * cfg.T * args.steps / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": f"{cfg.fmt} weights, bf16 activations, fp32 accumulate",
+        "data": "synthetic (seeded; shapes of the pages' model, random weights)",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "f": cfg.f, "n_shared": cfg.n_shared, "weights": f"{cfg.fmt} g{cfg.group}",
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {R} weight copies x {POOL} hidden batches cycled",
+                   "cuda_graph": graphs is not None},
+        "roofline": {"bound": "hbm", "kernel": "grouped gate/up + SwiGLU",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "avg_launch_ms": gu_avg_ms,
+                     "layer_frac": float(np.mean(layer_bytes)) / (ms_per_step * 1e-3) / 1e9 / peak},
+        "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
+        "gpu_launches": launches_per_step(cfg.T, cfg.k) * args.steps,
+        "clocks": clk.summary(),
+        "device_status": status,
+    }
+    return res, L, cfg
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    cfg = synth.CONFIGS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        L = synth.make_layer(cfg, routed=synth.make_bank(cfg, "routed", experts=[]),
+                             shared=synth.make_bank(cfg, "shared"))
+        # only the experts the sampled tokens touch are drawn (others are never read)
+        from oracle import moe_oracle as O
+        need = np.unique(O.select_topk(O.router_logits(L.x[:64], L.router_w, L.router_bias),
+                                       cfg.k)[0])
+        L.routed = synth.make_bank(cfg, "routed", experts=need)
+        rate, cores, sample = cpu_oracle_rate(cfg, L, args.cpu_seconds)
+        line = {"impl": "reference", "metric": f"MoE-layer tokens/s ({cfg.name}, T={cfg.T})",
+                "value": rate, "unit": "tokens/s", "n_gpus": 0, "steps": args.steps,
+                "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": cfg.name, "T": cfg.T},
+                "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores,
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    res, L, cfg = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1:
+        rate, cores, sample = cpu_oracle_rate(cfg, L, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(res))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

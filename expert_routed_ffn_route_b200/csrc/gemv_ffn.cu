@@ -1,0 +1,432 @@
+// Grouped expert FFN for few rows per expert (decode and verify calls, 1..32 tokens):
+// split-K, bandwidth-bound GEMV kernels over the touched experts only.
+//
+// Work unit = (active expert, 32 weight rows). A 256-thread CTA owns one unit at a time:
+// warps 0-3 take rows 0-15, warps 4-7 rows 16-31, and within each half the four warps
+// split the K groups round-robin; partial sums are added in a fixed order (no atomics),
+// so results do not depend on scheduling. Weights stream straight from HBM into registers
+// with 128-bit non-allocating loads (each expert row is read once per 8-token chunk), and
+// the products run on the tensor cores with mma.sync m16n8k16 (bf16 in, fp32 out): the
+// weights are the 16-row A operand, up to 8 tokens are the N = 8 B operand.
+//
+// The group scale multiplies the fp32 partial of its 128-wide K group, so quantised codes
+// enter the tensor core exactly (integers |q| <= 127 are exact in bf16).
+//
+// int4 codes are widened with a bf16 bit trick: the nibble n (after flipping its sign bit,
+// u = n ^ 8 = q + 8) is placed in the low mantissa bits of 128.0 (0x4300), giving the exact
+// bf16 value 128 + u = q + 136; the constant 136 * sum(x over the group) is subtracted from
+// each group's partial afterwards.
+//
+// What each part computes: gate/up kernel h = silu(Wg x) * (Wu x) for every grouped row
+// (Qwen3.8-Flash-Next-Dual-GPU README, "Dedicated prefill lane", step 2: grouped W4/W8-A16
+// products on the tensor cores); down kernel y = Wd h into one fp32 row per assignment
+// (same section, step 4). Unselected experts are never read (TandemLLM docs,
+// "17 Qwen3.8-Flash-Next", §17.4).
+#include <mutex>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kTok = 8;       // tokens per MMA (N)
+constexpr int kRowsCTA = 32;  // weight rows per CTA
+constexpr int kKSplit = 4;    // warps sharing one 16-row tile along K
+constexpr int kThreads = 256;
+
+template <int FMT> struct FmtInfo;
+template <> struct FmtInfo<4> { static constexpr int U = 1; static constexpr int bits = 4; };
+template <> struct FmtInfo<8> { static constexpr int U = 2; static constexpr int bits = 8; };
+template <> struct FmtInfo<16> { static constexpr int U = 4; static constexpr int bits = 16; };
+
+// Physical 8-byte unit of logical unit u inside a staged activation row. The XOR spreads
+// the four lanes of a quad over distinct banks; together with a row stride of 2K + 8 bytes
+// every half-warp's 8-byte reads are conflict free.
+__device__ __forceinline__ int phys_unit(int u) { return u ^ (((u >> 4) & 1) << 2); }
+
+__device__ __forceinline__ void mma_bf16_16x8x16(float (&c)[4], uint32_t a0, uint32_t a1,
+                                                 uint32_t a2, uint32_t a3, uint32_t b0,
+                                                 uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));  // (a&b)|c
+  return r;
+}
+
+// A fragments of one weight row for the 8 MMAs of a 128-wide K group.
+// fr[m][0] holds the pair for virtual k (2q, 2q+1), fr[m][1] for (2q+8, 2q+9).
+template <int FMT>
+__device__ __forceinline__ void to_frags(const uint4 (&raw)[FmtInfo<FMT>::U], uint32_t (&fr)[8][2]);
+
+template <>
+__device__ __forceinline__ void to_frags<4>(const uint4 (&raw)[1], uint32_t (&fr)[8][2]) {
+  const uint32_t w[4] = {raw[0].x ^ 0x88888888u, raw[0].y ^ 0x88888888u,
+                         raw[0].z ^ 0x88888888u, raw[0].w ^ 0x88888888u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    fr[2 * i][0] = lop_and_or(w[i], 0x000F000Fu, 0x43004300u);        // nibbles 0, 4
+    fr[2 * i][1] = lop_and_or(w[i] >> 4, 0x000F000Fu, 0x43004300u);   // nibbles 1, 5
+    fr[2 * i + 1][0] = lop_and_or(w[i] >> 8, 0x000F000Fu, 0x43004300u);  // 2, 6
+    fr[2 * i + 1][1] = lop_and_or(w[i] >> 12, 0x000F000Fu, 0x43004300u); // 3, 7
+  }
+}
+
+__device__ __forceinline__ uint32_t i8pair_to_bf16x2(uint32_t w, int lo_byte) {
+  const float a = static_cast<float>(static_cast<int8_t>((w >> (8 * lo_byte)) & 0xff));
+  const float b = static_cast<float>(static_cast<int8_t>((w >> (8 * lo_byte + 8)) & 0xff));
+  return pack_bf16x2(a, b);  // exact: |q| <= 127
+}
+
+template <>
+__device__ __forceinline__ void to_frags<8>(const uint4 (&raw)[2], uint32_t (&fr)[8][2]) {
+  const uint32_t w[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w,
+                         raw[1].x, raw[1].y, raw[1].z, raw[1].w};
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    fr[m][0] = i8pair_to_bf16x2(w[m], 0);
+    fr[m][1] = i8pair_to_bf16x2(w[m], 2);
+  }
+}
+
+template <>
+__device__ __forceinline__ void to_frags<16>(const uint4 (&raw)[4], uint32_t (&fr)[8][2]) {
+  const uint32_t w[16] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y,
+                          raw[1].z, raw[1].w, raw[2].x, raw[2].y, raw[2].z, raw[2].w,
+                          raw[3].x, raw[3].y, raw[3].z, raw[3].w};
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    fr[m][0] = w[2 * m];
+    fr[m][1] = w[2 * m + 1];
+  }
+}
+
+// One staged 16-byte chunk (8 bf16 of an activation row) in the order the A fragments use:
+// int4 pairs nibble i with nibble i + 4 inside each 8-wide word, so the chunk is stored as
+// elements (0,4,1,5,2,6,3,7); the other formats keep the natural order.
+template <int FMT>
+__device__ __forceinline__ void permute_chunk(uint4& v) {
+  if constexpr (FMT == 4) {
+    const uint32_t a = v.x, b = v.y, c = v.z, d = v.w;  // (0,1) (2,3) (4,5) (6,7)
+    v.x = __byte_perm(a, c, 0x5410);  // 0, 4
+    v.y = __byte_perm(a, c, 0x7632);  // 1, 5
+    v.z = __byte_perm(b, d, 0x5410);  // 2, 6
+    v.w = __byte_perm(b, d, 0x7632);  // 3, 7
+  }
+}
+
+struct StageArgs {
+  const uint16_t* src;   // activation rows (bf16)
+  int src_stride;        // elements between rows
+  const int32_t* perm;   // grouped row -> assignment (routed gate/up) or NULL
+  int k;                 // routed experts a token (assignment -> token)
+  int row0, nrows;       // rows [row0, row0 + nrows) of this chunk (grouped numbering)
+};
+
+// Stage up to 8 activation rows into shared memory (and per-group sums for int4).
+template <int FMT>
+__device__ void stage_rows(const StageArgs& a, int K, uint8_t* xs, int S, float* xsum) {
+  const int chunks = K / 8;  // 16-byte chunks per row
+  const int G = K / kGroup;
+  for (int i = threadIdx.x; i < kTok * chunks; i += kThreads) {
+    const int row = i / chunks, c = i % chunks;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row < a.nrows) {
+      int src_row = a.row0 + row;
+      if (a.perm) src_row = a.perm[src_row] / a.k;
+      v = *reinterpret_cast<const uint4*>(a.src + (size_t)src_row * a.src_stride + 8 * c);
+    }
+    if constexpr (FMT == 4) {
+      // fixed-order sum of the chunk, then over the 16 chunks of the group (a half-warp)
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        s += __uint_as_float(vv[q] << 16);
+        s += __uint_as_float(vv[q] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if ((c & 15) == 0) xsum[row * G + c / 16] = s;
+    }
+    permute_chunk<FMT>(v);
+    uint8_t* rowp = xs + (size_t)row * S;
+    *reinterpret_cast<uint2*>(rowp + 8 * phys_unit(2 * c)) = make_uint2(v.x, v.y);
+    *reinterpret_cast<uint2*>(rowp + 8 * phys_unit(2 * c + 1)) = make_uint2(v.z, v.w);
+  }
+}
+
+// Per-CTA view of one unit.
+struct Unit {
+  int e;          // expert index within its bank
+  bool shared;
+  int row_begin;  // first grouped row (routed) / first token (shared)
+  int nrows;
+  int tile;       // 32-row tile of the weight matrix
+};
+
+__device__ __forceinline__ bool get_unit(const Plan& p, int u, int n_tiles, Unit& out) {
+  const int n_active = p.active[0];
+  const int slot = u / n_tiles;
+  out.tile = u % n_tiles;
+  if (slot < n_active) {
+    out.e = p.active[1 + slot];
+    out.shared = false;
+    out.row_begin = p.offsets[out.e];
+    out.nrows = p.offsets[out.e + 1] - out.row_begin;
+    return true;
+  }
+  if (slot == n_active && p.has_shared) {
+    out.e = 0;
+    out.shared = true;
+    out.row_begin = 0;
+    out.nrows = p.T;
+    return true;
+  }
+  return false;
+}
+
+// Multiply one K group: NM matrices (gate+up or down) on the 8 staged tokens.
+template <int FMT, int NM>
+__device__ __forceinline__ void group_mma(const uint4 (&ra)[NM][FmtInfo<FMT>::U],
+                                          const uint4 (&rb)[NM][FmtInfo<FMT>::U],
+                                          const float (&sa)[NM], const float (&sb)[NM],
+                                          const uint8_t* xrow, const float* xsum, int G, int g,
+                                          int q4, float (&acc)[NM][4]) {
+  uint32_t fa[NM][8][2], fb[NM][8][2];
+#pragma unroll
+  for (int mi = 0; mi < NM; ++mi) {
+    to_frags<FMT>(ra[mi], fa[mi]);
+    to_frags<FMT>(rb[mi], fb[mi]);
+  }
+  float c[NM][4];
+#pragma unroll
+  for (int mi = 0; mi < NM; ++mi)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[mi][i] = 0.f;
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const uint2 b = *reinterpret_cast<const uint2*>(xrow + 8 * phys_unit(32 * g + 8 * q4 + m));
+#pragma unroll
+    for (int mi = 0; mi < NM; ++mi)
+      mma_bf16_16x8x16(c[mi], fa[mi][m][0], fb[mi][m][0], fa[mi][m][1], fb[mi][m][1], b.x, b.y);
+  }
+  float corr0 = 0.f, corr1 = 0.f;
+  if constexpr (FMT == 4) {
+    corr0 = 136.f * xsum[(2 * q4) * G + g];
+    corr1 = 136.f * xsum[(2 * q4 + 1) * G + g];
+  }
+#pragma unroll
+  for (int mi = 0; mi < NM; ++mi) {
+    acc[mi][0] = fmaf(sa[mi], c[mi][0] - corr0, acc[mi][0]);
+    acc[mi][1] = fmaf(sa[mi], c[mi][1] - corr1, acc[mi][1]);
+    acc[mi][2] = fmaf(sb[mi], c[mi][2] - corr0, acc[mi][2]);
+    acc[mi][3] = fmaf(sb[mi], c[mi][3] - corr1, acc[mi][3]);
+  }
+}
+
+// GATE_UP: weights gate+up [f][d], activations x (gathered by perm), output h (bf16).
+// !GATE_UP: weights down [d][f], activations h, output y (fp32).
+template <int FMT, bool GATE_UP>
+__global__ void __launch_bounds__(kThreads) gemv_ffn_kernel(Plan p) {
+  constexpr int NM = GATE_UP ? 2 : 1;
+  constexpr int U = FmtInfo<FMT>::U;
+  constexpr int PF = (FMT == 4) ? 5 : (FMT == 8 ? (GATE_UP ? 3 : 4) : 2);
+  const int K = GATE_UP ? p.d : p.f;
+  const int N = GATE_UP ? p.f : p.d;
+  const int G = K / kGroup;
+  const int S = 2 * K + 8;
+  const int n_tiles = N / kRowsCTA;
+  const size_t row_bytes = (size_t)K * FmtInfo<FMT>::bits / 8;
+  const size_t mat_bytes = row_bytes * N;
+
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t* xs = smem;
+  float* xsum = reinterpret_cast<float*>(smem + kTok * S);
+  float* red = xsum + kTok * G;  // [8 warps][32 lanes][NM*4]
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rt = warp / kKSplit, ks = warp % kKSplit;
+  const int grp = lane >> 2, q4 = lane & 3;
+
+  for (int u = blockIdx.x;; u += gridDim.x) {
+    Unit un;
+    if (!get_unit(p, u, n_tiles, un)) break;
+    const Bank& bank = un.shared ? p.shared : p.routed;
+    const int ra_row = un.tile * kRowsCTA + rt * 16 + grp;
+    const int rb_row = ra_row + 8;
+    const uint8_t* wbase[NM];
+    const uint16_t* sbase[NM];
+#pragma unroll
+    for (int mi = 0; mi < NM; ++mi) {
+      const int which = GATE_UP ? mi : 2;
+      wbase[mi] = static_cast<const uint8_t*>(bank.w[which]) + (size_t)un.e * mat_bytes;
+      sbase[mi] = bank.s[which] ? bank.s[which] + ((size_t)un.e * N) * G : nullptr;
+    }
+    for (int c0 = 0; c0 < un.nrows; c0 += kTok) {
+      const int nr = min(kTok, un.nrows - c0);
+      StageArgs sa;
+      if (GATE_UP) {
+        sa.src = p.x;
+        sa.src_stride = p.d;
+        sa.perm = un.shared ? nullptr : p.perm;
+        sa.k = p.k;
+        sa.row0 = un.row_begin + c0;
+      } else {
+        sa.src = p.h;
+        sa.src_stride = p.f;
+        sa.perm = nullptr;
+        sa.k = 1;
+        sa.row0 = (un.shared ? p.T * p.k : 0) + un.row_begin + c0;
+      }
+      sa.nrows = nr;
+      __syncthreads();  // previous chunk's readers are done with xs / red
+      stage_rows<FMT>(sa, K, xs, S, xsum);
+      __syncthreads();
+
+      float acc[NM][4];
+#pragma unroll
+      for (int mi = 0; mi < NM; ++mi)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[mi][i] = 0.f;
+      const uint8_t* xrow = xs + (size_t)grp * S;
+
+      for (int gb = ks; gb < G; gb += kKSplit * PF) {
+        uint4 wa[PF][NM][U], wb[PF][NM][U];
+        float fsa[PF][NM], fsb[PF][NM];
+#pragma unroll
+        for (int pf = 0; pf < PF; ++pf) {
+          const int g = gb + kKSplit * pf;
+          if (g < G) {
+#pragma unroll
+            for (int mi = 0; mi < NM; ++mi) {
+              const uint8_t* pa = wbase[mi] + (size_t)ra_row * row_bytes +
+                                  (size_t)g * (kGroup * FmtInfo<FMT>::bits / 8) + q4 * (16 * U);
+              const uint8_t* pb = pa + 8 * row_bytes;
+#pragma unroll
+              for (int uu = 0; uu < U; ++uu) {
+                wa[pf][mi][uu] = ld_nc_v4(pa + 16 * uu);
+                wb[pf][mi][uu] = ld_nc_v4(pb + 16 * uu);
+              }
+              if (sbase[mi]) {
+                fsa[pf][mi] = bf16_to_f32(__ldg(sbase[mi] + (size_t)ra_row * G + g));
+                fsb[pf][mi] = bf16_to_f32(__ldg(sbase[mi] + (size_t)rb_row * G + g));
+              } else {
+                fsa[pf][mi] = 1.f;
+                fsb[pf][mi] = 1.f;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int pf = 0; pf < PF; ++pf) {
+          const int g = gb + kKSplit * pf;
+          if (g < G)
+            group_mma<FMT, NM>(wa[pf], wb[pf], fsa[pf], fsb[pf], xrow, xsum, G, g, q4, acc);
+        }
+      }
+      // fixed-order reduction over the K split
+      float* myred = red + ((size_t)warp * 32 + lane) * (NM * 4);
+#pragma unroll
+      for (int mi = 0; mi < NM; ++mi)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) myred[mi * 4 + i] = acc[mi][i];
+      __syncthreads();
+      if (ks == 0) {
+        float tot[NM][4];
+#pragma unroll
+        for (int mi = 0; mi < NM; ++mi)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tot[mi][i] = 0.f;
+        for (int s = 0; s < kKSplit; ++s) {
+          const float* r = red + ((size_t)(rt * kKSplit + s) * 32 + lane) * (NM * 4);
+#pragma unroll
+          for (int mi = 0; mi < NM; ++mi)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tot[mi][i] += r[mi * 4 + i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tok = 2 * q4 + (i & 1);
+          const int row = (i < 2) ? ra_row : rb_row;
+          if (tok >= nr) continue;
+          if constexpr (GATE_UP) {
+            const float g = tot[0][i], up = tot[1][i];
+            const float hval = g / (1.f + expf(-g)) * up;
+            const size_t hrow = (un.shared ? (size_t)p.T * p.k : 0) + un.row_begin + c0 + tok;
+            p.h[hrow * p.f + row] = f32_to_bf16_rn(hval);
+          } else {
+            float* dst = un.shared ? p.y_shared + (size_t)(un.row_begin + c0 + tok) * p.d
+                                   : p.y_assign + (size_t)(un.row_begin + c0 + tok) * p.d;
+            dst[row] = tot[0][i];
+          }
+        }
+      }
+    }
+  }
+}
+
+// Per-instantiation launch facts (dynamic shared memory opt-in, resident CTAs per SM),
+// settled on the first call so that later calls (and stream captures) make no attribute
+// or occupancy queries.
+struct LaunchCache {
+  std::mutex mu;
+  size_t smem = 0;
+  int per_sm = 0, sms = 0;
+};
+
+template <int FMT, bool GATE_UP>
+static cudaError_t launch_one(const Plan& p, cudaStream_t st) {
+  const int K = GATE_UP ? p.d : p.f;
+  const int N = GATE_UP ? p.f : p.d;
+  const int NM = GATE_UP ? 2 : 1;
+  const size_t smem = (size_t)kTok * (2 * K + 8) + sizeof(float) * kTok * (K / kGroup) +
+                      sizeof(float) * 8 * 32 * NM * 4;
+  auto kern = gemv_ffn_kernel<FMT, GATE_UP>;
+  static LaunchCache cache;
+  int per_sm, sms;
+  {
+    std::lock_guard<std::mutex> lock(cache.mu);
+    if (smem > cache.smem) {
+      cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+      if (err != cudaSuccess) return err;
+      int dev = 0;
+      if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+      if ((err = cudaDeviceGetAttribute(&cache.sms, cudaDevAttrMultiProcessorCount, dev)) !=
+          cudaSuccess)
+        return err;
+      if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cache.per_sm, kern, kThreads,
+                                                               smem)) != cudaSuccess)
+        return err;
+      cache.smem = smem;
+    }
+    per_sm = std::max(1, cache.per_sm);
+    sms = cache.sms;
+  }
+  const int max_slots = std::min(p.E, p.T * p.k) + (p.has_shared ? 1 : 0);
+  const long long units = (long long)max_slots * (N / kRowsCTA);
+  const int grid = (int)std::max(1LL, std::min<long long>(units, (long long)per_sm * sms));
+  kern<<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <bool GATE_UP>
+static cudaError_t launch_fmt(const Plan& p, cudaStream_t st) {
+  // both banks share one format (checked on the host)
+  switch (p.routed.fmt) {
+    case 4: return launch_one<4, GATE_UP>(p, st);
+    case 8: return launch_one<8, GATE_UP>(p, st);
+    default: return launch_one<16, GATE_UP>(p, st);
+  }
+}
+
+cudaError_t launch_gemv_gate_up(const Plan& p, cudaStream_t st) { return launch_fmt<true>(p, st); }
+cudaError_t launch_gemv_down(const Plan& p, cudaStream_t st) { return launch_fmt<false>(p, st); }
+
+}  // namespace moe

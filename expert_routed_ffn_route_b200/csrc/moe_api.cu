@@ -1,0 +1,302 @@
+// C ABI of the MoE FFN layer: host-side validation, workspace layout and kernel sequencing.
+// Every entry point validates its arguments before enqueuing anything and reports errors
+// as a moe_status; nothing here allocates, frees or synchronises on the compute path.
+#include <cstring>
+
+#include "common.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool bank_ok(const moe_bank& b, int expect_n, int d, int f) {
+  if (b.n_exp != expect_n) return false;
+  if (expect_n == 0) return true;
+  if (b.fmt != MOE_W_BF16 && b.fmt != MOE_W_INT8 && b.fmt != MOE_W_INT4) return false;
+  const void* w[3] = {b.w_gate, b.w_up, b.w_down};
+  for (const void* p : w)
+    if (!p || !aligned(p, 16)) return false;
+  if (b.fmt == MOE_W_BF16) return true;
+  if (b.group != kGroup) return false;
+  const void* s[3] = {b.s_gate, b.s_up, b.s_down};
+  for (const void* p : s)
+    if (!p || !aligned(p, 2)) return false;
+  (void)d;
+  (void)f;
+  return true;
+}
+
+moe_status validate(const moe_layer* L) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  if (L->T < 1 || L->d < 128 || L->f < 128 || L->E < 1 || L->k < 1) return MOE_ERR_INVALID_ARG;
+  if (L->d % 128 || L->f % 128) return MOE_ERR_INVALID_ARG;
+  if (L->d > 8192 || L->f > 8192) return MOE_ERR_UNSUPPORTED;
+  if (L->E > kMaxE || L->k > kMaxK || L->k > L->E) return MOE_ERR_UNSUPPORTED;
+  if ((long long)L->T * L->k > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
+  if (L->path < MOE_PATH_AUTO || L->path > MOE_PATH_TC) return MOE_ERR_INVALID_ARG;
+  if (!L->router_w || !aligned(L->router_w, 16)) return MOE_ERR_INVALID_ARG;
+  if (L->router_bias && !aligned(L->router_bias, 4)) return MOE_ERR_INVALID_ARG;
+  if (!bank_ok(L->routed, L->E, L->d, L->f)) return MOE_ERR_INVALID_ARG;
+  if (L->shared.n_exp != 0 && L->shared.n_exp != 1) return MOE_ERR_UNSUPPORTED;
+  if (!bank_ok(L->shared, L->shared.n_exp, L->d, L->f)) return MOE_ERR_INVALID_ARG;
+  if (L->shared.n_exp == 1 && L->shared.fmt != L->routed.fmt) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Workspace layout (offsets from the 256-byte aligned base).
+struct WsLayout {
+  size_t status, logits, topk_idx, topk_w, offsets, perm, inv, active, cta_hist, h, y_assign,
+      y_shared, total;
+};
+
+WsLayout layout(const moe_layer* L) {
+  WsLayout w{};
+  const size_t T = L->T, k = L->k, E = L->E, d = L->d, f = L->f;
+  const size_t n = T * k;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  w.status = take(kAlign);
+  w.logits = take(T * E * sizeof(float));
+  w.topk_idx = take(n * sizeof(int32_t));
+  w.topk_w = take(n * sizeof(float));
+  w.offsets = take((E + 1) * sizeof(int32_t));
+  w.perm = take(n * sizeof(int32_t));
+  w.inv = take(n * sizeof(int32_t));
+  w.active = take((E + 2) * sizeof(int32_t));
+  w.cta_hist = take((size_t)perm_chunks(L->T, L->k) * E * sizeof(int32_t));
+  w.h = take((n + T) * f * sizeof(uint16_t));
+  w.y_assign = take(n * d * sizeof(float));
+  w.y_shared = take(T * d * sizeof(float));
+  w.total = o;
+  return w;
+}
+
+Bank to_bank(const moe_bank& b) {
+  Bank r;
+  r.fmt = b.fmt;
+  r.w[0] = b.w_gate;
+  r.w[1] = b.w_up;
+  r.w[2] = b.w_down;
+  r.s[0] = static_cast<const uint16_t*>(b.s_gate);
+  r.s[1] = static_cast<const uint16_t*>(b.s_up);
+  r.s[2] = static_cast<const uint16_t*>(b.s_down);
+  if (b.fmt == MOE_W_BF16) r.s[0] = r.s[1] = r.s[2] = nullptr;
+  return r;
+}
+
+moe_status check_ws(const moe_layer* L, void* ws, size_t ws_bytes) {
+  if (!ws || !aligned(ws, kAlign)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < layout(L).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+Plan make_plan(const moe_layer* L, void* ws) {
+  const WsLayout w = layout(L);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  Plan p{};
+  p.T = L->T;
+  p.d = L->d;
+  p.f = L->f;
+  p.E = L->E;
+  p.k = L->k;
+  p.has_shared = L->shared.n_exp;
+  p.router_w = static_cast<const uint16_t*>(L->router_w);
+  p.router_bias = L->router_bias;
+  p.routed = to_bank(L->routed);
+  p.shared = to_bank(L->shared);
+  p.status = reinterpret_cast<int32_t*>(b + w.status);
+  p.logits = reinterpret_cast<float*>(b + w.logits);
+  p.topk_idx = reinterpret_cast<int32_t*>(b + w.topk_idx);
+  p.topk_w = reinterpret_cast<float*>(b + w.topk_w);
+  p.offsets = reinterpret_cast<int32_t*>(b + w.offsets);
+  p.perm = reinterpret_cast<int32_t*>(b + w.perm);
+  p.inv = reinterpret_cast<int32_t*>(b + w.inv);
+  p.active = reinterpret_cast<int32_t*>(b + w.active);
+  p.cta_hist = reinterpret_cast<int32_t*>(b + w.cta_hist);
+  p.h = reinterpret_cast<uint16_t*>(b + w.h);
+  p.y_assign = reinterpret_cast<float*>(b + w.y_assign);
+  p.y_shared = reinterpret_cast<float*>(b + w.y_shared);
+  return p;
+}
+
+#define MOE_TRY(expr)                                  \
+  do {                                                 \
+    cudaError_t _e = (expr);                           \
+    if (_e != cudaSuccess) return MOE_ERR_CUDA;        \
+  } while (0)
+
+moe_status run_ffn(const Plan& p, cudaStream_t st, void* const* marks, int n_marks) {
+  MOE_TRY(launch_gemv_gate_up(p, st));
+  if (n_marks > 3 && marks[3]) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(marks[3]), st));
+  MOE_TRY(launch_gemv_down(p, st));
+  if (n_marks > 4 && marks[4]) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(marks[4]), st));
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_str(int32_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_DEVICE: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+moe_status moe_validate(const moe_layer* L) { return validate(L); }
+
+size_t moe_workspace_size(const moe_layer* L) {
+  if (validate(L) != MOE_OK) return 0;
+  return layout(L).total;
+}
+
+moe_status moe_route(const moe_layer* L, const void* x, int32_t* topk_idx, float* topk_w,
+                     void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (!x || !aligned(x, 16) || !topk_idx || !topk_w || !aligned(topk_idx, 4) ||
+      !aligned(topk_w, 4))
+    return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, ws, ws_bytes)) != MOE_OK) return s;
+  Plan p = make_plan(L, ws);
+  p.x = static_cast<const uint16_t*>(x);
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_w;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  MOE_TRY(launch_router(p, st));
+  MOE_TRY(launch_topk(p, st));
+  return MOE_OK;
+}
+
+moe_status moe_permute(const moe_layer* L, const int32_t* topk_idx, int32_t* expert_offsets,
+                       int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (!topk_idx || !expert_offsets || !perm || !inv || !aligned(topk_idx, 4) ||
+      !aligned(expert_offsets, 4) || !aligned(perm, 4) || !aligned(inv, 4))
+    return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, ws, ws_bytes)) != MOE_OK) return s;
+  Plan p = make_plan(L, ws);
+  p.topk_idx = const_cast<int32_t*>(topk_idx);
+  p.offsets = expert_offsets;
+  p.perm = perm;
+  p.inv = inv;
+  MOE_TRY(launch_permute(p, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_grouped_ffn(const moe_layer* L, const void* x, const int32_t* expert_offsets,
+                           const int32_t* perm, float* y_assign, float* y_shared, void* ws,
+                           size_t ws_bytes, moe_stream_t stream) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (!x || !aligned(x, 16) || !expert_offsets || !perm || !y_assign || !aligned(y_assign, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (L->shared.n_exp && (!y_shared || !aligned(y_shared, 16))) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, ws, ws_bytes)) != MOE_OK) return s;
+  Plan p = make_plan(L, ws);
+  p.x = static_cast<const uint16_t*>(x);
+  p.offsets = const_cast<int32_t*>(expert_offsets);
+  p.perm = const_cast<int32_t*>(perm);
+  p.y_assign = y_assign;
+  if (y_shared) p.y_shared = y_shared;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  MOE_TRY(launch_schedule_from_offsets(p, st));
+  return run_ffn(p, st, nullptr, 0);
+}
+
+moe_status moe_combine(const moe_layer* L, const float* y_assign, const float* y_shared,
+                       const int32_t* inv, const float* topk_w, void* out,
+                       moe_stream_t stream) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (!y_assign || !aligned(y_assign, 16) || !inv || !topk_w || !out || !aligned(out, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (L->shared.n_exp && (!y_shared || !aligned(y_shared, 16))) return MOE_ERR_INVALID_ARG;
+  Plan p{};
+  p.T = L->T;
+  p.d = L->d;
+  p.k = L->k;
+  p.has_shared = L->shared.n_exp;
+  p.y_assign = const_cast<float*>(y_assign);
+  p.y_shared = const_cast<float*>(y_shared);
+  p.inv = const_cast<int32_t*>(inv);
+  p.topk_w = const_cast<float*>(topk_w);
+  MOE_TRY(launch_combine(p, out, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, void* out,
+                                    int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                                    int32_t* perm, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream, void* const* marks, int32_t n_marks) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (!x || !aligned(x, 16) || !out || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+  if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
+      (expert_offsets && !aligned(expert_offsets, 4)) || (perm && !aligned(perm, 4)))
+    return MOE_ERR_INVALID_ARG;
+  if (n_marks < 0 || (n_marks > 0 && !marks)) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, ws, ws_bytes)) != MOE_OK) return s;
+  Plan p = make_plan(L, ws);
+  p.x = static_cast<const uint16_t*>(x);
+  if (topk_idx) p.topk_idx = topk_idx;
+  if (topk_w) p.topk_w = topk_w;
+  if (expert_offsets) p.offsets = expert_offsets;
+  if (perm) p.perm = perm;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> cudaError_t {
+    if (i < n_marks && marks[i]) return cudaEventRecord(static_cast<cudaEvent_t>(marks[i]), st);
+    return cudaSuccess;
+  };
+  MOE_TRY(mark(0));
+  MOE_TRY(launch_router(p, st));
+  MOE_TRY(launch_topk(p, st));
+  MOE_TRY(mark(1));
+  MOE_TRY(launch_permute(p, st));
+  MOE_TRY(mark(2));
+  if ((s = run_ffn(p, st, marks, n_marks)) != MOE_OK) return s;
+  MOE_TRY(launch_combine(p, out, st));
+  MOE_TRY(mark(5));
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_layer* L, const void* x, void* out, int32_t* topk_idx,
+                             float* topk_w, int32_t* expert_offsets, int32_t* perm, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  return moe_layer_forward_marked(L, x, out, topk_idx, topk_w, expert_offsets, perm, ws,
+                                  ws_bytes, stream, nullptr, 0);
+}
+
+moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,
+                             moe_stream_t stream) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (!code) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, ws, ws_bytes)) != MOE_OK) return s;
+  int32_t* dev = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + layout(L).status);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  MOE_TRY(cudaMemcpyAsync(&h, dev, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  MOE_TRY(cudaStreamSynchronize(st));
+  MOE_TRY(cudaMemsetAsync(dev, 0, sizeof(int32_t), st));
+  *code = (h == DEV_OK) ? MOE_OK : (h == DEV_TIMEOUT ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE);
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,172 @@
+/*
+ * moe_b200.h — C ABI of the expert-routed MoE FFN layer for NVIDIA B200 (sm_100a).
+ *
+ * One call of the layer maps hidden states X [T, d] to the FFN output [T, d]:
+ *   route    logits = X Wr^T (+ b) in fp32; per token the k largest logits, ties to
+ *            the lower expert index, in rank order; gates = softmax over the k selected
+ *            logits. (Qwen3.8-Flash-Next-Dual-GPU README, "Independent decode lane": the
+ *            512-expert router uses a deterministic stable top-k; "Model artifact and
+ *            memory placement": the router is kept in BF16/F32.)
+ *   permute  an expert-major plan of the T*k assignments a = t*k + j: counts per expert,
+ *            their exclusive scan, and a stable scatter (experts ascending, tokens
+ *            ascending within an expert). (Same README, "Dedicated prefill lane", step 1;
+ *            TandemLLM docs, "17 Qwen3.8-Flash-Next", §17.4: rows sorted by expert, one
+ *            matrix product over each expert's rows.)
+ *   grouped FFN  for every grouped row r of expert e: h = silu(Wg_e x) * (Wu_e x),
+ *            y = Wd_e h, with group-quantised weights W = q * s (symmetric W4/W8, groups
+ *            of 128 along K, BF16 scales: README, "Model artifact and memory placement").
+ *            Unselected experts are never read (TandemLLM docs §17.4).
+ *   combine  out_t = sum_{j<k} gate[t,j] * y[inv[t*k+j]] + y_shared[t], summed in that
+ *            fixed order in fp32, rounded once to bf16, no atomics (README, "Dedicated
+ *            prefill lane", step 5). The shared expert runs on every token with weight 1
+ *            (TandemLLM docs Table 17.1: 10 routed and 1 shared run a token).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise, 16-byte aligned,
+ *     row-major, owned by the caller. The library never allocates device memory, never
+ *     frees, and never synchronises the stream on the compute path.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *   - Arguments are validated on the host before anything is enqueued; an invalid call
+ *     returns a negative moe_status and enqueues nothing. No call throws across the ABI.
+ *   - bf16 values are IEEE bfloat16 bit patterns (uint16).
+ *   - Weight encodings (bank.fmt):
+ *       MOE_W_BF16  W[e][n][k] bf16; scales unused (NULL).
+ *       MOE_W_INT8  W[e][n][k] int8 (symmetric, code range -127..127), scales bf16
+ *                   S[e][n][k / group].
+ *       MOE_W_INT4  W[e][n][k / 8] uint32, 8 two's-complement nibbles per word along K,
+ *                   element k at bits 4 * (k % 8) of word k / 8; scales as for int8.
+ *     gate and up are [n_exp][f][d] (N = f, K = d); down is [n_exp][d][f] (N = d, K = f).
+ *   - Supported shapes: 1 <= T, d % 128 == 0, f % 128 == 0, 1 <= k <= min(E, 32),
+ *     1 <= E <= 1024, group == 128 for the integer formats, shared.n_exp in {0, 1}.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1, /* a pointer, size, alignment or shape is not accepted   */
+  MOE_ERR_UNSUPPORTED = -2, /* a valid request this build does not implement         */
+  MOE_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch or attribute)       */
+  MOE_ERR_TIMEOUT = -4,     /* a bounded device-side wait gave up (device status)     */
+  MOE_ERR_WORKSPACE = -5,   /* workspace NULL, misaligned or smaller than required    */
+  MOE_ERR_DEVICE = -6       /* a device-side check failed (see moe_device_status)     */
+} moe_status;
+
+typedef enum { MOE_W_BF16 = 16, MOE_W_INT8 = 8, MOE_W_INT4 = 4 } moe_wfmt;
+
+/* Which grouped-FFN kernels run. AUTO picks the tensor-core (tcgen05) grouped GEMMs
+ * for large token counts and the split-K GEMV kernels for 1..32-row calls. */
+typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC = 2 } moe_path;
+
+/* One expert bank of n_exp experts (the routed bank has n_exp = E; the shared bank has
+ * n_exp = 0 or 1). Pointers are device pointers; experts are contiguous, expert e's
+ * slice starts at e * (N * K * bits / 8) bytes. */
+typedef struct {
+  int32_t fmt;   /* moe_wfmt */
+  int32_t group; /* 128 for MOE_W_INT8 / MOE_W_INT4; ignored for MOE_W_BF16 */
+  int32_t n_exp;
+  int32_t reserved;
+  const void* w_gate; /* [n_exp][f][d] encoded */
+  const void* w_up;   /* [n_exp][f][d] encoded */
+  const void* w_down; /* [n_exp][d][f] encoded */
+  const void* s_gate; /* bf16 [n_exp][f][d / group] or NULL (bf16 weights) */
+  const void* s_up;   /* bf16 [n_exp][f][d / group] or NULL */
+  const void* s_down; /* bf16 [n_exp][d][f / group] or NULL */
+} moe_bank;
+
+/* The layer: shapes, router and the two banks. Read by every call; not retained. */
+typedef struct {
+  int32_t T, d, f, E, k;
+  int32_t path;              /* moe_path */
+  const void* router_w;      /* bf16 [E][d] */
+  const float* router_bias;  /* fp32 [E] added to the logits, or NULL */
+  moe_bank routed;           /* n_exp == E */
+  moe_bank shared;           /* n_exp == 0 (no shared expert) or 1 */
+} moe_layer;
+
+/* ABI version of the loaded library (MOE_ABI_VERSION). */
+MOE_API int32_t moe_abi_version(void);
+
+/* Human-readable name of a status code. Never NULL; the string is static. */
+MOE_API const char* moe_status_str(int32_t status);
+
+/* Host-side validation of a layer descriptor (no CUDA call is made).
+ * Returns MOE_OK or MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED. */
+MOE_API moe_status moe_validate(const moe_layer* L);
+
+/* Bytes of device workspace every call on this layer needs (0 if L is invalid).
+ * The workspace is caller-owned, 256-byte aligned, and may be reused between calls
+ * that are ordered on one stream; concurrent calls need separate workspaces. */
+MOE_API size_t moe_workspace_size(const moe_layer* L);
+
+/* Route: topk_idx int32 [T][k] (expert ids, rank order) and topk_w fp32 [T][k]
+ * (gates, each row sums to 1). x: bf16 [T][d]. */
+MOE_API moe_status moe_route(const moe_layer* L, const void* x, int32_t* topk_idx, float* topk_w,
+                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Permute: from topk_idx [T][k], writes expert_offsets int32 [E + 1] (exclusive scan of
+ * the per-expert counts; offsets[E] = T * k), perm int32 [T * k] (perm[r] = assignment
+ * t * k + j at grouped row r) and inv int32 [T * k] (inv[t * k + j] = its grouped row). */
+MOE_API moe_status moe_permute(const moe_layer* L, const int32_t* topk_idx, int32_t* expert_offsets,
+                       int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Grouped FFN over the plan: y_assign fp32 [T * k][d] in grouped row order (row r is
+ * expert e's output for assignment perm[r], e such that offsets[e] <= r < offsets[e+1]),
+ * and y_shared fp32 [T][d] (the shared expert on every token; may be NULL only when
+ * shared.n_exp == 0). x: bf16 [T][d]. */
+MOE_API moe_status moe_grouped_ffn(const moe_layer* L, const void* x, const int32_t* expert_offsets,
+                           const int32_t* perm, float* y_assign, float* y_shared, void* ws,
+                           size_t ws_bytes, moe_stream_t stream);
+
+/* Combine: out bf16 [T][d] = sum_{j<k} topk_w[t][j] * y_assign[inv[t*k+j]] (+ y_shared[t]),
+ * accumulated in fp32 in the order j = 0..k-1, then the shared term; one rounding. */
+MOE_API moe_status moe_combine(const moe_layer* L, const float* y_assign, const float* y_shared,
+                       const int32_t* inv, const float* topk_w, void* out,
+                       moe_stream_t stream);
+
+/* The whole layer in one call: out bf16 [T][d] from x bf16 [T][d]. The optional outputs
+ * (topk_idx [T][k], topk_w [T][k], expert_offsets [E+1], perm [T*k]) are written when
+ * non-NULL. Intermediates live in the workspace. */
+MOE_API moe_status moe_layer_forward(const moe_layer* L, const void* x, void* out, int32_t* topk_idx,
+                             float* topk_w, int32_t* expert_offsets, int32_t* perm, void* ws,
+                             size_t ws_bytes, moe_stream_t stream);
+
+/* Stage marks for profiling: the same computation as moe_layer_forward, and each non-NULL
+ * entry of `marks` (cudaEvent_t handles created by the caller) is recorded on `stream`:
+ * marks[0] before the first kernel, marks[1] after routing, marks[2] after the plan,
+ * marks[3] after the gate/up kernel, marks[4] after the down kernel, marks[5] after the
+ * combine. n_marks may be smaller than MOE_N_MARKS; missing entries are skipped. */
+#define MOE_N_MARKS 6
+MOE_API moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, void* out,
+                                    int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                                    int32_t* perm, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream, void* const* marks, int32_t n_marks);
+
+/* Reads the device status word kept in the workspace (synchronises `stream`), writes
+ * the code to *code (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE) and clears it. */
+MOE_API moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,
+                             moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

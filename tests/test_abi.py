@@ -1,0 +1,89 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+validates descriptors on the host (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from expert_routed_ffn_route_b200 import _build, binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return binding.load_library()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_exports_match_header(lib):
+    names = header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(binding.EXPORTS)
+    assert lib.moe_abi_version() == 1
+
+
+def _desc(**kw):
+    fake = 1 << 20  # aligned non-NULL host-side stand-ins: validation never dereferences
+    bank = lambda n, fmt=4: binding.MoeBank(fmt, 128, n, 0, fake, fake, fake, fake, fake, fake)
+    d = binding.MoeLayer(16, 2560, 1024, 512, 10, 0, fake, None, bank(512), bank(1))
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("T", 0, -1), ("d", 100, -1), ("f", 130, -1), ("k", 0, -1), ("k", 33, -2),
+    ("E", 2048, -2), ("path", 7, -1), ("router_w", None, -1), ("router_w", (1 << 20) + 2, -1),
+])
+def test_validation_codes(lib, field, value, code):
+    d = _desc(**{field: value})
+    assert lib.moe_validate(ctypes.byref(d)) == code
+    assert lib.moe_workspace_size(ctypes.byref(d)) == 0
+
+
+def test_validation_banks(lib):
+    d = _desc()
+    assert lib.moe_validate(ctypes.byref(d)) == 0
+    d.routed.group = 64
+    assert lib.moe_validate(ctypes.byref(d)) == -1
+    d = _desc()
+    d.shared.n_exp = 2
+    assert lib.moe_validate(ctypes.byref(d)) == -2
+    d = _desc()
+    d.shared.fmt = 8
+    assert lib.moe_validate(ctypes.byref(d)) == -2
+    d = _desc()
+    d.routed.s_up = None
+    assert lib.moe_validate(ctypes.byref(d)) == -1
+    d = _desc()
+    d.routed.fmt = 16
+    d.routed.s_gate = d.routed.s_up = d.routed.s_down = None
+    d.shared.fmt = 16
+    assert lib.moe_validate(ctypes.byref(d)) == 0
+
+
+def test_workspace_size_grows_with_T(lib):
+    a = lib.moe_workspace_size(ctypes.byref(_desc(T=1)))
+    b = lib.moe_workspace_size(ctypes.byref(_desc(T=4096)))
+    assert 0 < a < b
+    assert a % 256 == 0 and b % 256 == 0
+
+
+def test_calls_reject_bad_arguments_before_any_cuda_call(lib):
+    d = _desc()
+    # NULL workspace / NULL x: rejected on the host, nothing enqueued
+    assert lib.moe_layer_forward(ctypes.byref(d), 1 << 20, 1 << 20, None, None, None, None,
+                                 None, 0, None) == -5
+    assert lib.moe_layer_forward(ctypes.byref(d), None, 1 << 20, None, None, None, None,
+                                 1 << 20, 1 << 40, None) == -1
+    assert lib.moe_route(None, None, None, None, None, 0, None) == -1
+    assert lib.moe_status_str(-4) == b"device-side wait timed out"

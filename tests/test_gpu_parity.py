@@ -1,0 +1,178 @@
+"""Parity of the CUDA library (called through the C ABI) against the fp64 oracle.
+
+Bar: expert indices, the plan (offsets, perm, inv) bit-exact; gates within 1e-5;
+the bf16 layer output within max|d| <= 1e-2 * rms(oracle) + 1e-3 (the tolerance the
+workload states for fp32 accumulation); bitwise run-to-run determinism.
+"""
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+from expert_routed_ffn_route_b200 import synth
+from conftest import bank_dict
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+GATE_TOL = 1e-5
+
+
+def out_tol(ref):
+    return 1e-2 * float(np.sqrt(np.mean(ref ** 2))) + 1e-3
+
+
+def to_dev_x(x_bits):
+    return torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def bf16_to_np(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.fixture(scope="module")
+def B():
+    from expert_routed_ffn_route_b200 import binding
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    binding.load_library()
+    return binding
+
+
+def oracle_run(L: synth.LayerInputs, tokens=None, x=None):
+    x = L.x if x is None else x
+    return O.layer_forward(x, L.router_w, L.router_bias, bank_dict(L.routed),
+                           bank_dict(L.shared), L.cfg.k, tokens=tokens)
+
+
+def check_layer(B, dl, L, x_bits, path, sample=None, check_stages=True):
+    T = x_bits.shape[0]
+    desc = dl.descriptor(T, path)
+    ws = B.alloc_workspace(desc)
+    x = to_dev_x(x_bits)
+    idx = torch.empty((T, L.cfg.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, L.cfg.k), dtype=torch.float32, device="cuda")
+    offs = torch.empty(L.cfg.E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * L.cfg.k, dtype=torch.int32, device="cuda")
+    out = B.layer_forward(desc, x, ws, topk_idx=idx, topk_w=w, offsets=offs, perm=perm)
+    out2 = B.layer_forward(desc, x, ws)
+    torch.cuda.synchronize()
+    assert B.device_status(desc, ws) == 0
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16)), "not deterministic"
+
+    tokens = np.arange(T) if sample is None else np.asarray(sample)
+    ref = oracle_run(L, tokens=tokens, x=x_bits)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"]), "expert indices differ"
+    np.testing.assert_allclose(w.cpu().numpy(), ref["gates"], rtol=0, atol=GATE_TOL)
+    assert np.array_equal(offs.cpu().numpy(), ref["offsets"])
+    assert np.array_equal(perm.cpu().numpy(), ref["perm"])
+    got = O.widen_bf16(bf16_to_np(out))[tokens]
+    err = np.abs(got - ref["out"]).max()
+    assert err <= out_tol(ref["out"]), f"max|d| {err} > {out_tol(ref['out'])}"
+
+    if check_stages:
+        # the four stage entry points give the fused call's result bit for bit
+        i2, w2 = B.route(desc, x, ws)
+        o2, p2, inv2 = B.permute(desc, i2, ws)
+        ya, ys = B.grouped_ffn(desc, x, o2, p2, ws, has_shared=dl.has_shared)
+        out3 = B.combine(desc, ya, ys, inv2, w2)
+        torch.cuda.synchronize()
+        assert torch.equal(i2, idx) and torch.equal(w2, w)
+        assert torch.equal(o2, offs) and torch.equal(p2, perm)
+        assert np.array_equal(inv2.cpu().numpy(), ref["inv"])
+        assert torch.equal(out3.view(torch.int16), out.view(torch.int16))
+    return err
+
+
+# ------------------------------------------------------------------ small shapes
+
+@pytest.fixture(scope="module")
+def tiny(B):
+    L = synth.make_layer("tiny")
+    return L, B.DeviceLayer(L)
+
+
+@pytest.mark.parametrize("path", ["gemv"])
+def test_tiny_full(B, tiny, path):
+    L, dl = tiny
+    check_layer(B, dl, L, L.x, path)
+
+
+@pytest.mark.parametrize("T", [1, 3, 33])
+def test_tiny_ragged_T(B, tiny, T):
+    L, dl = tiny
+    x = synth.make_hidden(L.cfg, L.router_w, L.router_bias, T=T, stream=f"ragged{T}")
+    check_layer(B, dl, L, x, "gemv")
+
+
+@pytest.mark.parametrize("fmt", ["int4", "int8", "bf16"])
+@pytest.mark.parametrize("shared", [1, 0])
+def test_formats_small(B, fmt, shared):
+    cfg = synth.LayerConfig(f"small-{fmt}", T=40, d=384, E=12, k=3, f=256, n_shared=shared,
+                            fmt=fmt, seed=3)
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "gemv")
+
+
+def test_zipf_bias_and_k1(B):
+    cfg = synth.LayerConfig("bias-k1", T=50, d=256, E=20, k=1, f=128, fmt="int8", zipf_s=1.1,
+                            seed=5)
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "gemv")
+
+
+def test_all_experts_selected(B):
+    cfg = synth.LayerConfig("k=E", T=17, d=256, E=4, k=4, f=128, fmt="int4", seed=7)
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "gemv")
+
+
+def test_many_rows_per_expert(B):
+    """One expert gets most rows (more than one 8-token chunk, ragged tail)."""
+    cfg = synth.LayerConfig("hot", T=100, d=256, E=8, k=2, f=128, fmt="int4", zipf_s=3.0, seed=9)
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "gemv")
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+@pytest.fixture(scope="module")
+def int4_bank(B):
+    cfg = synth.CONFIGS["decode"]
+    routed = synth.make_bank(cfg, "routed")
+    shared = synth.make_bank(cfg, "shared")
+    return routed, shared
+
+
+@pytest.mark.parametrize("name,sample", [("decode", None), ("verify16", None),
+                                         ("verify32", [0, 7, 31]),
+                                         ("prefill", [0, 1, 255, 511])])
+def test_full_size_int4(B, int4_bank, name, sample):
+    cfg = synth.CONFIGS[name]
+    routed, shared = int4_bank
+    L = synth.make_layer(cfg, routed=routed, shared=shared)
+    dl = B.DeviceLayer(L)
+    check_layer(B, dl, L, L.x, "auto", sample=sample, check_stages=(cfg.T <= 32))
+
+
+def test_full_size_long_int8(B):
+    cfg = synth.CONFIGS["long"]
+    L = synth.make_layer(cfg)
+    dl = B.DeviceLayer(L)
+    check_layer(B, dl, L, L.x, "auto", sample=[0, 1, 2047, 4095], check_stages=False)
+
+
+# ------------------------------------------------------------------ errors
+
+def test_errors_reported(B, tiny):
+    L, dl = tiny
+    desc = dl.descriptor(8)
+    ws = B.alloc_workspace(desc)
+    x = to_dev_x(L.x[:8])
+    with pytest.raises(B.MoeError) as e:
+        B.layer_forward(desc, x, ws[1:])          # misaligned and too small
+    assert e.value.status == -5
+    bad = dl.descriptor(8)
+    bad.k = 0
+    with pytest.raises(B.MoeError) as e:
+        B.layer_forward(bad, x, ws)
+    assert e.value.status == -1
