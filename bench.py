@@ -249,6 +249,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
+        torch.cuda.nvtx.range_push("timed")
         with torch.cuda.stream(stream):
             t_start.record(stream)
             for i in range(args.steps):
@@ -258,6 +259,7 @@ def run_ours(args, rank, world, local_rank):
                     step(i, marks_for(i))
             t_end.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     ms = t_start.elapsed_time(t_end)

@@ -27,3 +27,22 @@ def bank_dict(bank):
 def tiny_layer():
     from expert_routed_ffn_route_b200 import synth
     return synth.make_layer("tiny")
+
+
+def bf16_half_ulp(v):
+    """Half a unit in the last place of bf16 at |v| (8 significant bits)."""
+    import numpy as np
+    a = np.maximum(np.abs(v), np.finfo(np.float32).tiny)
+    return np.ldexp(1.0, np.floor(np.log2(a)).astype(np.int64) - 8)
+
+
+def output_excess(got, ref):
+    """Per-element error of a bf16 output beyond its own rounding: |got - ref| minus half a
+    bf16 ulp at max(|got|, |ref|). The layer bound (1e-2 * rms(ref) + 1e-3) applies to this."""
+    import numpy as np
+    return np.abs(got - ref) - bf16_half_ulp(np.maximum(np.abs(got), np.abs(ref)))
+
+
+def out_tol(ref):
+    import numpy as np
+    return 1e-2 * float(np.sqrt(np.mean(ref ** 2))) + 1e-3

@@ -2,23 +2,21 @@
 
 Bar: expert indices, the plan (offsets, perm, inv) bit-exact; gates within 1e-5;
 the bf16 layer output within max|d| <= 1e-2 * rms(oracle) + 1e-3 (the tolerance the
-workload states for fp32 accumulation); bitwise run-to-run determinism.
+workload states for fp32 accumulation), counted beyond the output's own rounding to
+bf16 (half a bf16 ulp of the element, which alone exceeds the bound for |out| >= 2);
+bitwise run-to-run determinism.
 """
 import numpy as np
 import pytest
 
 from oracle import moe_oracle as O
 from expert_routed_ffn_route_b200 import synth
-from conftest import bank_dict
+from conftest import bank_dict, out_tol, output_excess
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 GATE_TOL = 1e-5
-
-
-def out_tol(ref):
-    return 1e-2 * float(np.sqrt(np.mean(ref ** 2))) + 1e-3
 
 
 def to_dev_x(x_bits):
@@ -66,8 +64,11 @@ def check_layer(B, dl, L, x_bits, path, sample=None, check_stages=True):
     assert np.array_equal(offs.cpu().numpy(), ref["offsets"])
     assert np.array_equal(perm.cpu().numpy(), ref["perm"])
     got = O.widen_bf16(bf16_to_np(out))[tokens]
-    err = np.abs(got - ref["out"]).max()
-    assert err <= out_tol(ref["out"]), f"max|d| {err} > {out_tol(ref['out'])}"
+    err = float(output_excess(got, ref["out"]).max())
+    raw = float(np.abs(got - ref["out"]).max())
+    print(f"[{L.cfg.name} T={T} {path}] max|d| {raw:.3e}, beyond bf16 rounding {err:.3e}, "
+          f"bound {out_tol(ref['out']):.3e}")
+    assert err <= out_tol(ref["out"]), f"max excess {err} > {out_tol(ref['out'])}"
 
     if check_stages:
         # the four stage entry points give the fused call's result bit for bit

@@ -272,3 +272,14 @@ def test_planted_mistakes_are_caught(monkeypatch, mistake):
                             lambda x, Wg, Wu, Wd: (O.silu(x @ Wg.T) * (x @ Wu.T)) @ Wd[::-1].T)
     with pytest.raises(AssertionError):
         _check_worked(O.layer_forward)
+
+
+def test_bf16_half_ulp_helper():
+    """The rounding allowance used by the parity tests equals the distance to the next
+    bf16 value / 2 (checked with torch's own bf16 rounding)."""
+    from conftest import bf16_half_ulp
+    v = np.array([1.0, 1.5, 1.99, 2.0, 3.9, 0.3, -0.7, 1e-3])
+    nxt = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16) + 1
+    gap = (nxt.view(torch.bfloat16).to(torch.float64) -
+           torch.from_numpy(v).to(torch.bfloat16).to(torch.float64)).abs().numpy()
+    assert np.array_equal(bf16_half_ulp(v), gap / 2)
