@@ -130,11 +130,24 @@ Plan make_plan(const moe_layer* L, void* ws) {
     if (_e != cudaSuccess) return MOE_ERR_CUDA;        \
   } while (0)
 
+// Records mark i on the stream. The external flag makes the record a node of its own when
+// the stream is being captured into a CUDA graph, so the mark also fires on every replay.
+cudaError_t record_mark(void* const* marks, int n_marks, int i, cudaStream_t st) {
+  if (i >= n_marks || !marks[i]) return cudaSuccess;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t err = cudaStreamIsCapturing(st, &cap);
+  if (err != cudaSuccess) return err;
+  cudaEvent_t ev = static_cast<cudaEvent_t>(marks[i]);
+  if (cap == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  return cudaEventRecord(ev, st);
+}
+
 moe_status run_ffn(const Plan& p, cudaStream_t st, void* const* marks, int n_marks) {
   MOE_TRY(launch_gemv_gate_up(p, st));
-  if (n_marks > 3 && marks[3]) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(marks[3]), st));
+  MOE_TRY(record_mark(marks, n_marks, 3, st));
   MOE_TRY(launch_gemv_down(p, st));
-  if (n_marks > 4 && marks[4]) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(marks[4]), st));
+  MOE_TRY(record_mark(marks, n_marks, 4, st));
   return MOE_OK;
 }
 
@@ -260,10 +273,7 @@ moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, void* out
   if (expert_offsets) p.offsets = expert_offsets;
   if (perm) p.perm = perm;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  auto mark = [&](int i) -> cudaError_t {
-    if (i < n_marks && marks[i]) return cudaEventRecord(static_cast<cudaEvent_t>(marks[i]), st);
-    return cudaSuccess;
-  };
+  auto mark = [&](int i) -> cudaError_t { return record_mark(marks, n_marks, i, st); };
   MOE_TRY(mark(0));
   MOE_TRY(launch_router(p, st));
   MOE_TRY(launch_topk(p, st));
