@@ -39,13 +39,15 @@ POOL = 64
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode", choices=list(synth.CONFIGS))
     ap.add_argument("--replicas", type=int, default=0, help="weight copies cycled (0: auto)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--stage-times", action="store_true",
+                    help="also report per-stage CUDA-event times (stage marks block overlap)")
     return ap.parse_args()
 
 
@@ -150,11 +152,6 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def launches_per_step(T, k):
-    # router, top-k, plan (1 kernel up to 1024 assignments, else 3), gate/up, down, combine
-    return 2 + (1 if T * k <= 1024 else 3) + 3
-
-
 def run_ours(args, rank, world, local_rank):
     import torch
     from expert_routed_ffn_route_b200 import binding as B
@@ -208,38 +205,57 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
-    n_cap = min(args.steps, R * 8)
+    n_mark = min(args.steps, 256)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(n_cap)]
+          for _ in range(n_mark)]
     for a, b in ev:  # torch creates the CUDA event on its first record
         a.record(stream)
         b.record(stream)
 
-    def step(i, marks=None):
+    def step(i, marked=False):
+        marks = None
+        if marked:
+            marks = [None] * B.N_MARKS
+            marks[2], marks[3] = ev[i % n_mark]
         B.layer_forward(descs[i % R], x_dev[i % POOL], ws, out=out, marks=marks, stream=stream)
-
-    def marks_for(i):
-        m = [None] * B.N_MARKS
-        m[2], m[3] = ev[i % n_cap]
-        return m
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            step(i, marks_for(i))
+            step(i)
     torch.cuda.synchronize()
 
-    graphs = None
+    # The K timed steps are captured once into CUDA graphs of up to G steps each (a
+    # decode step is a few microseconds of GPU work; per-step host launches would
+    # dominate). A second, shorter pass with stage marks around the gate/up kernel gives
+    # that kernel's launch duration from CUDA events.
+    G = 64
+    plain, marked = [], []
     if not args.no_graph:
-        graphs = []
-        for i in range(n_cap):
+        for a0 in range(0, args.steps, G):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                step(i, marks_for(i))
-            graphs.append(g)
-        with torch.cuda.stream(stream):
-            for g in graphs:
+                for i in range(a0, min(args.steps, a0 + G)):
+                    step(i)
+            plain.append(g)
+        for a0 in range(0, n_mark, G):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(a0, min(n_mark, a0 + G)):
+                    step(i, marked=True)
+            marked.append(g)
+        with torch.cuda.stream(stream):  # one untimed pass over every graph
+            for g in plain + marked:
                 g.replay()
         torch.cuda.synchronize()
+
+    def run(graphs, n, with_marks):
+        with torch.cuda.stream(stream):
+            if graphs:
+                for g in graphs:
+                    g.replay()
+            else:
+                for i in range(n):
+                    step(i, marked=with_marks)
 
     # ---- timed region
     t_start = torch.cuda.Event(enable_timing=True)
@@ -249,27 +265,43 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
+        time.sleep(0.3)  # let the sampler start before the timed region
         torch.cuda.nvtx.range_push("timed")
-        with torch.cuda.stream(stream):
-            t_start.record(stream)
-            for i in range(args.steps):
-                if graphs is not None:
-                    graphs[i % n_cap].replay()
-                else:
-                    step(i, marks_for(i))
-            t_end.record(stream)
+        t_start.record(stream)
+        run(plain, args.steps, False)
+        t_end.record(stream)
         torch.cuda.synchronize()
         torch.cuda.nvtx.range_pop()
     if world > 1:
         dist.barrier()
     ms = t_start.elapsed_time(t_end)
 
-    # dominant kernel: the captured steps' gate/up launches (the last replay of each graph)
-    last = range(max(0, args.steps - n_cap), args.steps)
-    k_ms = [ev[i % n_cap][0].elapsed_time(ev[i % n_cap][1]) for i in last]
-    k_bytes = [gu_bytes[i % POOL] for i in last]
+    # dominant kernel: gate/up launches of the marked pass (CUDA events on the launch stream)
+    torch.cuda.synchronize()
+    run(marked, n_mark, True)
+    torch.cuda.synchronize()
+    k_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n_mark)]
+    k_bytes = [gu_bytes[i % POOL] for i in range(n_mark)]
     gu_avg_ms = float(np.mean(k_ms))
     achieved = float(np.sum(k_bytes) / (np.sum(k_ms) * 1e-3) / 1e9)
+
+    stage_ms = None
+    if args.stage_times:
+        n_st = min(args.steps, 200)
+        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(B.N_MARKS)]
+               for _ in range(n_st)]
+        for row in sev:  # torch creates the CUDA event on its first record
+            for e_ in row:
+                e_.record(stream)
+        with torch.cuda.stream(stream):
+            for i in range(n_st):
+                B.layer_forward(descs[i % R], x_dev[i % POOL], ws, out=out, marks=sev[i],
+                                stream=stream)
+        torch.cuda.synchronize()
+        names = ["route", "plan", "gate_up", "down", "combine"]
+        stage_ms = {n: float(np.mean([sev[i][j].elapsed_time(sev[i][j + 1])
+                                      for i in range(n_st // 2, n_st)]))
+                    for j, n in enumerate(names)}
 
     # ---- end to end through the public call with host buffers
     x_host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -315,7 +347,7 @@ def run_ours(args, rank, world, local_rank):
                    "f": cfg.f, "n_shared": cfg.n_shared, "weights": f"{cfg.fmt} g{cfg.group}",
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {R} weight copies x {POOL} hidden batches cycled",
-                   "cuda_graph": graphs is not None},
+                   "cuda_graph": not args.no_graph},
         "roofline": {"bound": "hbm", "kernel": "grouped gate/up + SwiGLU",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
@@ -323,9 +355,10 @@ def run_ours(args, rank, world, local_rank):
                      "layer_frac": float(np.mean(layer_bytes)) / (ms_per_step * 1e-3) / 1e9 / peak},
         "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
-        "gpu_launches": launches_per_step(cfg.T, cfg.k) * args.steps,
+        "gpu_launches": B.launches_per_call(descs[0]) * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
+        **({"stages_ms_eager": stage_ms} if stage_ms else {}),
     }
     return res, L, cfg
 

@@ -44,7 +44,7 @@ class MoeLayer(ctypes.Structure):
 _LIB = None
 EXPORTS = ["moe_abi_version", "moe_status_str", "moe_validate", "moe_workspace_size",
            "moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
-           "moe_layer_forward_marked", "moe_device_status"]
+           "moe_layer_forward_marked", "moe_device_status", "moe_launches_per_call"]
 
 
 def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
@@ -74,6 +74,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "moe_layer_forward_marked": (I32, [LP, P, P, P, P, P, P, P, SZ, P,
                                            ctypes.POINTER(P), I32]),
         "moe_device_status": (I32, [LP, P, SZ, ctypes.POINTER(I32), P]),
+        "moe_launches_per_call": (I32, [LP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -234,6 +235,10 @@ def layer_forward(L: MoeLayer, x, ws, out=None, topk_idx=None, topk_w=None, offs
                                           _stream(stream), arr, len(marks))
     _check(st, "moe_layer_forward")
     return out
+
+
+def launches_per_call(L: MoeLayer) -> int:
+    return load_library().moe_launches_per_call(ctypes.byref(L))
 
 
 def device_status(L: MoeLayer, ws, stream=None) -> int:

@@ -44,6 +44,84 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, DEV_OK, code);
 }
 
+// ------------------------------------------------------------------ stable top-k
+
+// Order-preserving map of a finite float to uint32 (larger float -> larger key); -0 and
+// +0 map to the same key, so they tie like equal values do. key_value inverts it.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t b = __float_as_uint(v + 0.0f);  // -0 + 0 = +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// Warp-cooperative stable top-k of one row of E <= 32 * PER keys (order_key values): the k
+// largest, ties to the lower index, in rank order. Lane j < k ends with the j-th pick's index
+// in *idx and its key in *key. Lane l holds keys l, l + 32, ... in registers. Each round is
+// two warp reductions (the best key, then the lowest index holding it); only the lane that
+// owned the pick rescans its PER registers (no memory traffic inside the rounds).
+template <int PER>
+__device__ __forceinline__ void warp_topk_regs(const float* row, int E, int k, int lane, int* idx,
+                                               uint32_t* key) {
+  uint32_t kv[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    kv[i] = (e < E) ? order_key(__ldcg(row + e)) : 0u;  // 0: absent or taken
+  }
+  uint32_t bk = 0;
+  int bi = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i)
+    if (kv[i] > bk) {  // strict: the lowest index wins among this lane's equal keys
+      bk = kv[i];
+      bi = i;
+    }
+  *idx = 0;
+  *key = 0;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t mine = (bk == m && m != 0) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, mine);
+    if (lane == j) {
+      *idx = (int)win;
+      *key = m;
+    }
+    if (mine == win) {  // the owner retires its pick and finds its next best
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (i == bi) kv[i] = 0;
+      bk = 0;
+      bi = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (kv[i] > bk) {
+          bk = kv[i];
+          bi = i;
+        }
+    }
+  }
+}
+
+// Dispatch on the keys a lane holds (E <= 1024).
+__device__ __forceinline__ void warp_topk(const float* row, int E, int k, int lane, int* idx,
+                                          uint32_t* key) {
+  if (E <= 256) warp_topk_regs<8>(row, E, k, lane, idx, key);
+  else if (E <= 512) warp_topk_regs<16>(row, E, k, lane, idx, key);
+  else warp_topk_regs<32>(row, E, k, lane, idx, key);
+}
+
+// Gates of the k picks held by lanes 0..k-1: softmax of their logits, summed in rank order.
+__device__ __forceinline__ float warp_topk_gate(uint32_t my_key, uint32_t top_key, int k,
+                                                int lane) {
+  const float z = (lane < k) ? expf(key_value(my_key) - key_value(top_key)) : 0.f;
+  float total = 0.f;
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) total += __shfl_sync(0xffffffffu, z, j);
+  return z / total;
+}
+
 // ------------------------------------------------------------------ launch plumbing
 
 // Everything a kernel needs about one call, resolved on the host.
@@ -76,6 +154,21 @@ struct Plan {
   float* y_assign;     // [T*k*d]
   float* y_shared;     // [T*d]
   int32_t* status;
+  int32_t* ticket;     // zero between calls; the fused routing kernel's completion counter
+  uint16_t* xg;        // tensor-core path: x rows gathered into grouped order [T*k][d]
+  int32_t* tc_sched;   // tensor-core path: per-slot schedule (TcSched view)
+  int path;            // moe_path
+};
+
+// Per slot (active routed experts in ascending order, then the shared expert): rows, first
+// row, expert id (-1: shared) and the running count of 128-row m-tiles, written by
+// tc_prep_kernel. A GEMM with n_tiles weight tiles per expert has units
+// [mt_prefix[s] * n_tiles, mt_prefix[s + 1] * n_tiles) in slot s.
+struct TcSched {
+  int32_t* slot_rows;    // [E + 2]
+  int32_t* slot_row0;    // [E + 2]
+  int32_t* slot_expert;  // [E + 2]
+  int32_t* mt_prefix;    // [E + 2]; mt_prefix[n_slots] = total m-tiles
 };
 
 // Permutation chunking (assignments per scatter CTA).
@@ -89,6 +182,21 @@ cudaError_t launch_permute(const Plan& p, cudaStream_t st);
 cudaError_t launch_schedule_from_offsets(const Plan& p, cudaStream_t st);
 cudaError_t launch_gemv_gate_up(const Plan& p, cudaStream_t st);
 cudaError_t launch_gemv_down(const Plan& p, cudaStream_t st);
-cudaError_t launch_combine(const Plan& p, void* out, cudaStream_t st);
+cudaError_t launch_combine(const Plan& p, void* out, cudaStream_t st, bool pdl);
+// TMA-pipelined grouped GEMV (int4 weights, scales 16-byte aligned)
+bool tma_gemv_supported(const Plan& p);
+cudaError_t launch_tma_gate_up(const Plan& p, cudaStream_t st, bool pdl);
+cudaError_t launch_tma_down(const Plan& p, cudaStream_t st, bool pdl);
+// tcgen05 grouped GEMMs (tc_grouped.cu)
+bool tc_supported(const Plan& p);
+size_t tc_sched_bytes(int E);
+TcSched tc_sched_view(void* base, int E);
+cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st);
+cudaError_t launch_tc_gate_up(const Plan& p, const TcSched& S, const uint16_t* xg,
+                              cudaStream_t st);
+cudaError_t launch_tc_down(const Plan& p, const TcSched& S, cudaStream_t st);
+// router + top-k + plan in one launch (T <= 32)
+bool route_fused_supported(const Plan& p);
+cudaError_t launch_route_fused(const Plan& p, int32_t* ticket, cudaStream_t st);
 
 }  // namespace moe

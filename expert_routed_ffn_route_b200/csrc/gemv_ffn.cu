@@ -24,142 +24,13 @@
 // "17 Qwen3.8-Flash-Next", §17.4).
 #include <mutex>
 
-#include "common.cuh"
+#include "gemv_frag.cuh"
 
 namespace moe {
 
-constexpr int kTok = 8;       // tokens per MMA (N)
 constexpr int kRowsCTA = 32;  // weight rows per CTA
 constexpr int kKSplit = 4;    // warps sharing one 16-row tile along K
 constexpr int kThreads = 256;
-
-template <int FMT> struct FmtInfo;
-template <> struct FmtInfo<4> { static constexpr int U = 1; static constexpr int bits = 4; };
-template <> struct FmtInfo<8> { static constexpr int U = 2; static constexpr int bits = 8; };
-template <> struct FmtInfo<16> { static constexpr int U = 4; static constexpr int bits = 16; };
-
-// Physical 8-byte unit of logical unit u inside a staged activation row. The XOR spreads
-// the four lanes of a quad over distinct banks; together with a row stride of 2K + 8 bytes
-// every half-warp's 8-byte reads are conflict free.
-__device__ __forceinline__ int phys_unit(int u) { return u ^ (((u >> 4) & 1) << 2); }
-
-__device__ __forceinline__ void mma_bf16_16x8x16(float (&c)[4], uint32_t a0, uint32_t a1,
-                                                 uint32_t a2, uint32_t a3, uint32_t b0,
-                                                 uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));  // (a&b)|c
-  return r;
-}
-
-// A fragments of one weight row for the 8 MMAs of a 128-wide K group.
-// fr[m][0] holds the pair for virtual k (2q, 2q+1), fr[m][1] for (2q+8, 2q+9).
-template <int FMT>
-__device__ __forceinline__ void to_frags(const uint4 (&raw)[FmtInfo<FMT>::U], uint32_t (&fr)[8][2]);
-
-template <>
-__device__ __forceinline__ void to_frags<4>(const uint4 (&raw)[1], uint32_t (&fr)[8][2]) {
-  const uint32_t w[4] = {raw[0].x ^ 0x88888888u, raw[0].y ^ 0x88888888u,
-                         raw[0].z ^ 0x88888888u, raw[0].w ^ 0x88888888u};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    fr[2 * i][0] = lop_and_or(w[i], 0x000F000Fu, 0x43004300u);        // nibbles 0, 4
-    fr[2 * i][1] = lop_and_or(w[i] >> 4, 0x000F000Fu, 0x43004300u);   // nibbles 1, 5
-    fr[2 * i + 1][0] = lop_and_or(w[i] >> 8, 0x000F000Fu, 0x43004300u);  // 2, 6
-    fr[2 * i + 1][1] = lop_and_or(w[i] >> 12, 0x000F000Fu, 0x43004300u); // 3, 7
-  }
-}
-
-__device__ __forceinline__ uint32_t i8pair_to_bf16x2(uint32_t w, int lo_byte) {
-  const float a = static_cast<float>(static_cast<int8_t>((w >> (8 * lo_byte)) & 0xff));
-  const float b = static_cast<float>(static_cast<int8_t>((w >> (8 * lo_byte + 8)) & 0xff));
-  return pack_bf16x2(a, b);  // exact: |q| <= 127
-}
-
-template <>
-__device__ __forceinline__ void to_frags<8>(const uint4 (&raw)[2], uint32_t (&fr)[8][2]) {
-  const uint32_t w[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w,
-                         raw[1].x, raw[1].y, raw[1].z, raw[1].w};
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    fr[m][0] = i8pair_to_bf16x2(w[m], 0);
-    fr[m][1] = i8pair_to_bf16x2(w[m], 2);
-  }
-}
-
-template <>
-__device__ __forceinline__ void to_frags<16>(const uint4 (&raw)[4], uint32_t (&fr)[8][2]) {
-  const uint32_t w[16] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y,
-                          raw[1].z, raw[1].w, raw[2].x, raw[2].y, raw[2].z, raw[2].w,
-                          raw[3].x, raw[3].y, raw[3].z, raw[3].w};
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    fr[m][0] = w[2 * m];
-    fr[m][1] = w[2 * m + 1];
-  }
-}
-
-// One staged 16-byte chunk (8 bf16 of an activation row) in the order the A fragments use:
-// int4 pairs nibble i with nibble i + 4 inside each 8-wide word, so the chunk is stored as
-// elements (0,4,1,5,2,6,3,7); the other formats keep the natural order.
-template <int FMT>
-__device__ __forceinline__ void permute_chunk(uint4& v) {
-  if constexpr (FMT == 4) {
-    const uint32_t a = v.x, b = v.y, c = v.z, d = v.w;  // (0,1) (2,3) (4,5) (6,7)
-    v.x = __byte_perm(a, c, 0x5410);  // 0, 4
-    v.y = __byte_perm(a, c, 0x7632);  // 1, 5
-    v.z = __byte_perm(b, d, 0x5410);  // 2, 6
-    v.w = __byte_perm(b, d, 0x7632);  // 3, 7
-  }
-}
-
-struct StageArgs {
-  const uint16_t* src;   // activation rows (bf16)
-  int src_stride;        // elements between rows
-  const int32_t* perm;   // grouped row -> assignment (routed gate/up) or NULL
-  int k;                 // routed experts a token (assignment -> token)
-  int row0, nrows;       // rows [row0, row0 + nrows) of this chunk (grouped numbering)
-};
-
-// Stage up to 8 activation rows into shared memory (and per-group sums for int4).
-template <int FMT>
-__device__ void stage_rows(const StageArgs& a, int K, uint8_t* xs, int S, float* xsum) {
-  const int chunks = K / 8;  // 16-byte chunks per row
-  const int G = K / kGroup;
-  for (int i = threadIdx.x; i < kTok * chunks; i += kThreads) {
-    const int row = i / chunks, c = i % chunks;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (row < a.nrows) {
-      int src_row = a.row0 + row;
-      if (a.perm) src_row = a.perm[src_row] / a.k;
-      v = *reinterpret_cast<const uint4*>(a.src + (size_t)src_row * a.src_stride + 8 * c);
-    }
-    if constexpr (FMT == 4) {
-      // fixed-order sum of the chunk, then over the 16 chunks of the group (a half-warp)
-      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-      float s = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        s += __uint_as_float(vv[q] << 16);
-        s += __uint_as_float(vv[q] & 0xffff0000u);
-      }
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if ((c & 15) == 0) xsum[row * G + c / 16] = s;
-    }
-    permute_chunk<FMT>(v);
-    uint8_t* rowp = xs + (size_t)row * S;
-    *reinterpret_cast<uint2*>(rowp + 8 * phys_unit(2 * c)) = make_uint2(v.x, v.y);
-    *reinterpret_cast<uint2*>(rowp + 8 * phys_unit(2 * c + 1)) = make_uint2(v.z, v.w);
-  }
-}
 
 // Per-CTA view of one unit.
 struct Unit {
@@ -189,45 +60,6 @@ __device__ __forceinline__ bool get_unit(const Plan& p, int u, int n_tiles, Unit
     return true;
   }
   return false;
-}
-
-// Multiply one K group: NM matrices (gate+up or down) on the 8 staged tokens.
-template <int FMT, int NM>
-__device__ __forceinline__ void group_mma(const uint4 (&ra)[NM][FmtInfo<FMT>::U],
-                                          const uint4 (&rb)[NM][FmtInfo<FMT>::U],
-                                          const float (&sa)[NM], const float (&sb)[NM],
-                                          const uint8_t* xrow, const float* xsum, int G, int g,
-                                          int q4, float (&acc)[NM][4]) {
-  uint32_t fa[NM][8][2], fb[NM][8][2];
-#pragma unroll
-  for (int mi = 0; mi < NM; ++mi) {
-    to_frags<FMT>(ra[mi], fa[mi]);
-    to_frags<FMT>(rb[mi], fb[mi]);
-  }
-  float c[NM][4];
-#pragma unroll
-  for (int mi = 0; mi < NM; ++mi)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) c[mi][i] = 0.f;
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const uint2 b = *reinterpret_cast<const uint2*>(xrow + 8 * phys_unit(32 * g + 8 * q4 + m));
-#pragma unroll
-    for (int mi = 0; mi < NM; ++mi)
-      mma_bf16_16x8x16(c[mi], fa[mi][m][0], fb[mi][m][0], fa[mi][m][1], fb[mi][m][1], b.x, b.y);
-  }
-  float corr0 = 0.f, corr1 = 0.f;
-  if constexpr (FMT == 4) {
-    corr0 = 136.f * xsum[(2 * q4) * G + g];
-    corr1 = 136.f * xsum[(2 * q4 + 1) * G + g];
-  }
-#pragma unroll
-  for (int mi = 0; mi < NM; ++mi) {
-    acc[mi][0] = fmaf(sa[mi], c[mi][0] - corr0, acc[mi][0]);
-    acc[mi][1] = fmaf(sa[mi], c[mi][1] - corr1, acc[mi][1]);
-    acc[mi][2] = fmaf(sb[mi], c[mi][2] - corr0, acc[mi][2]);
-    acc[mi][3] = fmaf(sb[mi], c[mi][3] - corr1, acc[mi][3]);
-  }
 }
 
 // GATE_UP: weights gate+up [f][d], activations x (gathered by perm), output h (bf16).
@@ -286,7 +118,7 @@ __global__ void __launch_bounds__(kThreads) gemv_ffn_kernel(Plan p) {
       }
       sa.nrows = nr;
       __syncthreads();  // previous chunk's readers are done with xs / red
-      stage_rows<FMT>(sa, K, xs, S, xsum);
+      stage_rows<FMT, kThreads>(sa, K, xs, S, xsum, threadIdx.x);
       __syncthreads();
 
       float acc[NM][4];

@@ -1,0 +1,372 @@
+// Grouped expert FFN for few rows per expert (decode and verify calls) with int4 weights:
+// weight tiles move HBM -> shared memory through the TMA engine (one-dimensional bulk
+// copies) in a multi-stage mbarrier pipeline, and 8 consumer warps run the products on the
+// tensor cores (mma.sync m16n8k16, fragments from gemv_frag.cuh).
+//
+// Layout facts used: in the int4 encoding an expert matrix is row-major with K contiguous,
+// so ROWS consecutive rows of one expert form ONE contiguous block of ROWS * K / 2 bytes,
+// and their group scales [ROWS][K / 128] another. A stage is one such tile of every matrix
+// the kernel needs (gate and up for the first kernel, down for the second) plus scales; one
+// thread issues two bulk copies per matrix and the copies complete on the stage's mbarrier.
+//
+// Work: tiles (active expert, ROWS rows) in a flat list; CTA c (one per SM, persistent)
+// takes a contiguous range, so consecutive tiles mostly share an expert and its staged
+// activation rows. Each weight byte is read from HBM once per call; tokens beyond 8 for one
+// expert re-use the staged tile from shared memory.
+//
+// What is computed is the same as gemv_ffn.cu: h = silu(Wg x) * (Wu x) per grouped row
+// (Qwen3.8-Flash-Next-Dual-GPU README, "Dedicated prefill lane", step 2), then one fp32
+// y = Wd h per assignment (step 4); unselected experts are never read (TandemLLM docs,
+// "17 Qwen3.8-Flash-Next", §17.4).
+#include <mutex>
+
+#include "gemv_frag.cuh"
+#include "pipeline.cuh"
+
+namespace moe {
+
+#ifdef MOE_TRACE
+__device__ long long g_trace[2][160][64];
+#define TRACE(slot) \
+  do { if (ctid == 0 && blockIdx.x < 160 && (slot) < 64) g_trace[GATE_UP ? 0 : 1][blockIdx.x][(slot)] = clock64(); } while (0)
+#else
+#define TRACE(slot) do {} while (0)
+#endif
+
+constexpr int kCons = 16;                    // consumer warps
+constexpr int kTmaThreads = 32 * (kCons + 1);  // + one producer warp
+
+template <bool GATE_UP> struct TmaShape {
+  static constexpr int ROWS = GATE_UP ? 32 : 64;  // weight rows per tile
+  static constexpr int NM = GATE_UP ? 2 : 1;      // matrices per tile
+  static constexpr int RT = ROWS / 16;            // 16-row MMA tiles per tile
+  static constexpr int KS = kCons / RT;           // consumer warps sharing one row tile (K split)
+  static constexpr int NS = GATE_UP ? 2 : 5;      // pipeline stages
+};
+
+struct TmaSmem {
+  size_t stage_bytes, w_bytes, s_bytes, xs_off, xsum_off, red_off, bar_off, flag_off, total;
+};
+
+template <bool GATE_UP>
+__host__ __device__ inline TmaSmem tma_smem_layout(int K) {
+  using Sh = TmaShape<GATE_UP>;
+  TmaSmem m;
+  const int G = K / kGroup;
+  m.w_bytes = (size_t)Sh::ROWS * K / 2;        // one matrix tile (int4)
+  m.s_bytes = (size_t)Sh::ROWS * G * 2;        // its scales (bf16)
+  m.stage_bytes = Sh::NM * (m.w_bytes + m.s_bytes);
+  size_t o = Sh::NS * m.stage_bytes;
+  m.xs_off = o;
+  o += (size_t)kTok * (2 * K + 8);
+  o = (o + 15) & ~size_t(15);
+  m.xsum_off = o;
+  o += sizeof(float) * kTok * G;
+  m.red_off = o;
+  o += sizeof(float) * kCons * 32 * Sh::NM * 4;
+  o = (o + 15) & ~size_t(15);
+  m.bar_off = o;
+  o += sizeof(uint64_t) * 2 * Sh::NS;
+  m.flag_off = o;
+  o += 16;
+  m.total = o;
+  return m;
+}
+
+// Tile -> expert and rows. Slots 0..n_active-1 are the active routed experts (ascending
+// ids), slot n_active is the shared expert.
+struct TileInfo {
+  int slot, e, shared, row_begin, nrows, rowtile;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const Plan& p, int ti, int n_rowtiles,
+                                              int n_active) {
+  TileInfo t;
+  t.slot = ti / n_rowtiles;
+  t.rowtile = ti % n_rowtiles;
+  if (t.slot < n_active) {
+    t.e = p.active[1 + t.slot];
+    t.shared = 0;
+    t.row_begin = p.offsets[t.e];
+    t.nrows = p.offsets[t.e + 1] - t.row_begin;
+  } else {
+    t.e = 0;
+    t.shared = 1;
+    t.row_begin = 0;
+    t.nrows = p.T;
+  }
+  return t;
+}
+
+// Stage the activation rows of token chunk c0 of tile t (x gathered through perm for the
+// gate/up kernel, the h rows of the tile's expert for the down kernel).
+template <bool GATE_UP>
+__device__ __forceinline__ void stage_tile_rows(const Plan& p, const TileInfo& t, int c0, int K,
+                                                uint8_t* xs, int S, float* xsum, int ctid) {
+  StageArgs sa;
+  if (GATE_UP) {
+    sa.src = p.x;
+    sa.src_stride = p.d;
+    sa.perm = t.shared ? nullptr : p.perm;
+    sa.k = p.k;
+    sa.row0 = t.row_begin + c0;
+  } else {
+    sa.src = p.h;
+    sa.src_stride = p.f;
+    sa.perm = nullptr;
+    sa.k = 1;
+    sa.row0 = (t.shared ? p.T * p.k : 0) + t.row_begin + c0;
+  }
+  sa.nrows = min(kTok, t.nrows - c0);
+  stage_rows<4, 32 * kCons>(sa, K, xs, S, xsum, ctid);
+}
+
+template <bool GATE_UP>
+__global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
+  using Sh = TmaShape<GATE_UP>;
+  constexpr int NM = Sh::NM;
+  const int K = GATE_UP ? p.d : p.f;
+  const int N = GATE_UP ? p.f : p.d;
+  const int G = K / kGroup;
+  const int S = 2 * K + 8;
+  const size_t row_bytes = (size_t)K / 2;
+  const TmaSmem L = tma_smem_layout<GATE_UP>(K);
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* xs = smem + L.xs_off;
+  float* xsum = reinterpret_cast<float*>(smem + L.xsum_off);
+  float* red = reinterpret_cast<float*>(smem + L.red_off);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* empty = full + Sh::NS;
+  volatile int* flag = reinterpret_cast<volatile int*>(smem + L.flag_off);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#ifdef MOE_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 160) {
+    unsigned long long gt;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt));
+    g_trace[GATE_UP ? 0 : 1][blockIdx.x][61] = (long long)gt;
+    g_trace[GATE_UP ? 0 : 1][blockIdx.x][62] = clock64();
+  }
+#endif
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Sh::NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCons);
+    }
+    flag[0] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  KT_ENTRY(GATE_UP ? 2 : 3);
+  pdl_wait();     // plan and activations come from the preceding kernels
+  KT_READY(GATE_UP ? 2 : 3);
+
+  const int n_active = p.active[0];
+  const int n_rowtiles = N / Sh::ROWS;
+  const int n_tiles = (n_active + (p.has_shared ? 1 : 0)) * n_rowtiles;
+  const int t_begin = (int)((long long)n_tiles * blockIdx.x / gridDim.x);
+  const int t_end = (int)((long long)n_tiles * (blockIdx.x + 1) / gridDim.x);
+
+  if (warp == kCons) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int i = 0;
+      for (int ti = t_begin; ti < t_end; ++ti, ++i) {
+        const int s = i % Sh::NS, u = i / Sh::NS;
+        if (u > 0 && !mbar_wait(&empty[s], (u - 1) & 1)) {
+          set_status(p.status, DEV_TIMEOUT);
+          break;
+        }
+        const TileInfo t = tile_info(p, ti, n_rowtiles, n_active);
+        const Bank& bank = t.shared ? p.shared : p.routed;
+        uint8_t* st = smem + (size_t)s * L.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)L.stage_bytes);
+#pragma unroll
+        for (int mi = 0; mi < NM; ++mi) {
+          const int which = GATE_UP ? mi : 2;
+          const uint8_t* wsrc = static_cast<const uint8_t*>(bank.w[which]) +
+                                ((size_t)t.e * N + (size_t)t.rowtile * Sh::ROWS) * row_bytes;
+          const uint16_t* ssrc = bank.s[which] + ((size_t)t.e * N + (size_t)t.rowtile * Sh::ROWS) * G;
+          bulk_g2s(st + mi * L.w_bytes, wsrc, (uint32_t)L.w_bytes, &full[s]);
+          bulk_g2s(st + NM * L.w_bytes + mi * L.s_bytes, ssrc, (uint32_t)L.s_bytes, &full[s]);
+        }
+      }
+      // drain: every issued stage must land before the CTA may exit
+      const int issued = i;
+      for (int j = (issued > Sh::NS ? issued - Sh::NS : 0); j < issued; ++j)
+        mbar_wait(&full[j % Sh::NS], (j / Sh::NS) & 1);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int ctid = threadIdx.x;  // 0 .. 255
+#ifdef MOE_TRACE
+  int tr = 0;
+  TRACE(tr++);
+#endif
+  const int rt = warp / Sh::KS, ks = warp % Sh::KS;
+  const int grp = lane >> 2, q4 = lane & 3;
+  int staged_slot = -1, staged_c0 = -1;
+  int i = 0;
+  for (int ti = t_begin; ti < t_end; ++ti, ++i) {
+    const int s = i % Sh::NS, u = i / Sh::NS;
+    const TileInfo t = tile_info(p, ti, n_rowtiles, n_active);
+    // The first token chunk of a new expert is staged before the wait for the tile's
+    // weights, so the activation loads overlap the weight copies.
+    const bool pre = (staged_slot != t.slot || staged_c0 != 0);
+    if (pre) stage_tile_rows<GATE_UP>(p, t, 0, K, xs, S, xsum, ctid);
+    if (ctid == 0) flag[1] = mbar_wait(&full[s], u & 1) ? 1 : 0;
+#ifdef MOE_TRACE
+    TRACE(tr++);
+#endif
+    named_bar_sync(1, 32 * kCons);
+    if (!flag[1]) {
+      if (ctid == 0) set_status(p.status, DEV_TIMEOUT);
+      break;
+    }
+    if (pre) {
+      staged_slot = t.slot;
+      staged_c0 = 0;
+    }
+    const uint8_t* st = smem + (size_t)s * L.stage_bytes;
+    const int la = rt * 16 + grp, lb = la + 8;  // rows inside the tile
+
+    for (int c0 = 0; c0 < t.nrows; c0 += kTok) {
+      const int nr = min(kTok, t.nrows - c0);
+      if (staged_slot != t.slot || staged_c0 != c0) {
+        named_bar_sync(1, 32 * kCons);  // everyone is done with the previous rows
+        stage_tile_rows<GATE_UP>(p, t, c0, K, xs, S, xsum, ctid);
+        named_bar_sync(1, 32 * kCons);
+#ifdef MOE_TRACE
+        TRACE(tr++);
+#endif
+        staged_slot = t.slot;
+        staged_c0 = c0;
+      }
+      float acc[NM][4];
+#pragma unroll
+      for (int mi = 0; mi < NM; ++mi)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[mi][q] = 0.f;
+      const uint8_t* xrow = xs + (size_t)grp * S;
+      for (int g = ks; g < G; g += Sh::KS) {
+        uint4 wa[NM][1], wb[NM][1];
+        float fsa[NM], fsb[NM];
+#pragma unroll
+        for (int mi = 0; mi < NM; ++mi) {
+          const uint8_t* wt = st + mi * L.w_bytes;
+          wa[mi][0] = *reinterpret_cast<const uint4*>(wt + la * row_bytes + g * 64 + q4 * 16);
+          wb[mi][0] = *reinterpret_cast<const uint4*>(wt + lb * row_bytes + g * 64 + q4 * 16);
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + NM * L.w_bytes + mi * L.s_bytes);
+          fsa[mi] = bf16_to_f32(sc[la * G + g]);
+          fsb[mi] = bf16_to_f32(sc[lb * G + g]);
+        }
+        group_mma<4, NM>(wa, wb, fsa, fsb, xrow, xsum, G, g, q4, acc);
+      }
+      float* myred = red + ((size_t)warp * 32 + lane) * (NM * 4);
+#pragma unroll
+      for (int mi = 0; mi < NM; ++mi)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) myred[mi * 4 + q] = acc[mi][q];
+      TRACE(tr++);
+      named_bar_sync(1, 32 * kCons);
+      TRACE(tr++);
+      // fixed-order sum over the K split, then the epilogue
+      for (int o = ctid; o < Sh::ROWS * kTok; o += 32 * kCons) {
+        const int row = o / kTok, tok = o % kTok;
+        if (tok >= nr) continue;
+        const int rtile = row / 16, r16 = row % 16;
+        const int l = (r16 % 8) * 4 + tok / 2, q = (r16 / 8) * 2 + (tok % 2);
+        float tot[NM];
+#pragma unroll
+        for (int mi = 0; mi < NM; ++mi) tot[mi] = 0.f;
+        for (int k2 = 0; k2 < Sh::KS; ++k2) {
+          const float* r = red + ((size_t)(rtile * Sh::KS + k2) * 32 + l) * (NM * 4);
+#pragma unroll
+          for (int mi = 0; mi < NM; ++mi) tot[mi] += r[mi * 4 + q];
+        }
+        const int n = t.rowtile * Sh::ROWS + row;
+        if constexpr (GATE_UP) {
+          const float gte = tot[0], up = tot[1];
+          const float hval = gte / (1.f + expf(-gte)) * up;
+          const size_t hrow = (t.shared ? (size_t)p.T * p.k : 0) + t.row_begin + c0 + tok;
+          p.h[hrow * p.f + n] = f32_to_bf16_rn(hval);
+        } else {
+          float* dst = t.shared ? p.y_shared + (size_t)(c0 + tok) * p.d
+                                : p.y_assign + (size_t)(t.row_begin + c0 + tok) * p.d;
+          dst[n] = tot[0];
+        }
+      }
+      named_bar_sync(1, 32 * kCons);
+      TRACE(tr++);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+  if (ctid == 0) KT_EXIT(GATE_UP ? 2 : 3);
+  pdl_trigger();  // dependents start as this CTA finishes (see route_fused.cu)
+}
+
+struct TmaLaunchCache {
+  std::mutex mu;
+  size_t smem = 0;
+  int sms = 0;
+};
+
+template <bool GATE_UP>
+static cudaError_t launch_tma(const Plan& p, cudaStream_t st, bool pdl) {
+  const int K = GATE_UP ? p.d : p.f;
+  const size_t smem = tma_smem_layout<GATE_UP>(K).total;
+  auto kern = gemv_tma_kernel<GATE_UP>;
+  static TmaLaunchCache cache;
+  int sms;
+  {
+    std::lock_guard<std::mutex> lock(cache.mu);
+    if (smem > cache.smem) {
+      cudaError_t err =
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (err != cudaSuccess) return err;
+      int dev = 0;
+      if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+      if ((err = cudaDeviceGetAttribute(&cache.sms, cudaDevAttrMultiProcessorCount, dev)) !=
+          cudaSuccess)
+        return err;
+      cache.smem = smem;
+    }
+    sms = cache.sms;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(kTmaThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+#ifdef MOE_TRACE
+extern "C" __attribute__((visibility("default"))) int moe_trace_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_trace, sizeof(g_trace));
+}
+#endif
+
+bool tma_gemv_supported(const Plan& p) {
+  if (p.routed.fmt != 4) return false;
+  return tma_smem_layout<true>(p.d).total <= 227 * 1024 &&
+         tma_smem_layout<false>(p.f).total <= 227 * 1024;
+}
+
+cudaError_t launch_tma_gate_up(const Plan& p, cudaStream_t st, bool pdl) {
+  return launch_tma<true>(p, st, pdl);
+}
+cudaError_t launch_tma_down(const Plan& p, cudaStream_t st, bool pdl) {
+  return launch_tma<false>(p, st, pdl);
+}
+
+}  // namespace moe

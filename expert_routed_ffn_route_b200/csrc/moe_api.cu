@@ -51,7 +51,7 @@ moe_status validate(const moe_layer* L) {
 // Workspace layout (offsets from the 256-byte aligned base).
 struct WsLayout {
   size_t status, logits, topk_idx, topk_w, offsets, perm, inv, active, cta_hist, h, y_assign,
-      y_shared, total;
+      y_shared, xg, tc_sched, total;
 };
 
 WsLayout layout(const moe_layer* L) {
@@ -72,6 +72,8 @@ WsLayout layout(const moe_layer* L) {
   w.h = take((n + T) * f * sizeof(uint16_t));
   w.y_assign = take(n * d * sizeof(float));
   w.y_shared = take(T * d * sizeof(float));
+  w.xg = take(n * d * sizeof(uint16_t));
+  w.tc_sched = take(tc_sched_bytes(L->E));
   w.total = o;
   return w;
 }
@@ -110,6 +112,7 @@ Plan make_plan(const moe_layer* L, void* ws) {
   p.routed = to_bank(L->routed);
   p.shared = to_bank(L->shared);
   p.status = reinterpret_cast<int32_t*>(b + w.status);
+  p.ticket = reinterpret_cast<int32_t*>(b + w.status + 16);
   p.logits = reinterpret_cast<float*>(b + w.logits);
   p.topk_idx = reinterpret_cast<int32_t*>(b + w.topk_idx);
   p.topk_w = reinterpret_cast<float*>(b + w.topk_w);
@@ -121,6 +124,9 @@ Plan make_plan(const moe_layer* L, void* ws) {
   p.h = reinterpret_cast<uint16_t*>(b + w.h);
   p.y_assign = reinterpret_cast<float*>(b + w.y_assign);
   p.y_shared = reinterpret_cast<float*>(b + w.y_shared);
+  p.xg = reinterpret_cast<uint16_t*>(b + w.xg);
+  p.tc_sched = reinterpret_cast<int32_t*>(b + w.tc_sched);
+  p.path = L->path;
   return p;
 }
 
@@ -143,11 +149,58 @@ cudaError_t record_mark(void* const* marks, int n_marks, int i, cudaStream_t st)
   return cudaEventRecord(ev, st);
 }
 
+bool scales_aligned16(const Bank& b) {
+  for (int i = 0; i < 3; ++i)
+    if (b.s[i] && !aligned(b.s[i], 16)) return false;
+  return true;
+}
+
+// Grouped FFN kernels for the call: the TMA-pipelined GEMV for int4 banks, the
+// register-streaming GEMV otherwise. Kernels after the first of a call use programmatic
+// dependent launch (their prologue overlaps the tail of the previous kernel).
+// Tensor-core grouped GEMMs for calls with more than 32 tokens (or when asked for).
+bool use_tc(const Plan& p) {
+  if (p.path == MOE_PATH_GEMV) return false;
+  if (p.path == MOE_PATH_TC) return true;
+  return p.T > 32;
+}
+
 moe_status run_ffn(const Plan& p, cudaStream_t st, void* const* marks, int n_marks) {
-  MOE_TRY(launch_gemv_gate_up(p, st));
-  MOE_TRY(record_mark(marks, n_marks, 3, st));
-  MOE_TRY(launch_gemv_down(p, st));
+  if (use_tc(p)) {
+    if (!tc_supported(p)) return MOE_ERR_UNSUPPORTED;
+    const TcSched S = tc_sched_view(p.tc_sched, p.E);
+    MOE_TRY(launch_tc_prep(p, S, p.xg, st));
+    MOE_TRY(launch_tc_gate_up(p, S, p.xg, st));
+    MOE_TRY(record_mark(marks, n_marks, 3, st));
+    MOE_TRY(launch_tc_down(p, S, st));
+    MOE_TRY(record_mark(marks, n_marks, 4, st));
+    return MOE_OK;
+  }
+  const bool tma = tma_gemv_supported(p) && scales_aligned16(p.routed) &&
+                   (!p.has_shared || scales_aligned16(p.shared));
+  if (tma) {
+    MOE_TRY(launch_tma_gate_up(p, st, true));
+    MOE_TRY(record_mark(marks, n_marks, 3, st));
+    MOE_TRY(launch_tma_down(p, st, true));
+  } else {
+    MOE_TRY(launch_gemv_gate_up(p, st));
+    MOE_TRY(record_mark(marks, n_marks, 3, st));
+    MOE_TRY(launch_gemv_down(p, st));
+  }
   MOE_TRY(record_mark(marks, n_marks, 4, st));
+  return MOE_OK;
+}
+
+// Routing (+ the plan when the fused kernel applies). Returns whether the plan is done.
+moe_status run_route(const Plan& p, cudaStream_t st, bool* plan_done) {
+  if (route_fused_supported(p)) {
+    MOE_TRY(launch_route_fused(p, p.ticket, st));
+    *plan_done = true;
+  } else {
+    MOE_TRY(launch_router(p, st));
+    MOE_TRY(launch_topk(p, st));
+    *plan_done = false;
+  }
   return MOE_OK;
 }
 
@@ -190,9 +243,8 @@ moe_status moe_route(const moe_layer* L, const void* x, int32_t* topk_idx, float
   p.topk_idx = topk_idx;
   p.topk_w = topk_w;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  MOE_TRY(launch_router(p, st));
-  MOE_TRY(launch_topk(p, st));
-  return MOE_OK;
+  bool plan_done = false;
+  return run_route(p, st, &plan_done);
 }
 
 moe_status moe_permute(const moe_layer* L, const int32_t* topk_idx, int32_t* expert_offsets,
@@ -250,7 +302,7 @@ moe_status moe_combine(const moe_layer* L, const float* y_assign, const float* y
   p.y_shared = const_cast<float*>(y_shared);
   p.inv = const_cast<int32_t*>(inv);
   p.topk_w = const_cast<float*>(topk_w);
-  MOE_TRY(launch_combine(p, out, reinterpret_cast<cudaStream_t>(stream)));
+  MOE_TRY(launch_combine(p, out, reinterpret_cast<cudaStream_t>(stream), false));
   return MOE_OK;
 }
 
@@ -275,13 +327,13 @@ moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, void* out
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> cudaError_t { return record_mark(marks, n_marks, i, st); };
   MOE_TRY(mark(0));
-  MOE_TRY(launch_router(p, st));
-  MOE_TRY(launch_topk(p, st));
+  bool plan_done = false;
+  if ((s = run_route(p, st, &plan_done)) != MOE_OK) return s;
   MOE_TRY(mark(1));
-  MOE_TRY(launch_permute(p, st));
+  if (!plan_done) MOE_TRY(launch_permute(p, st));
   MOE_TRY(mark(2));
   if ((s = run_ffn(p, st, marks, n_marks)) != MOE_OK) return s;
-  MOE_TRY(launch_combine(p, out, st));
+  MOE_TRY(launch_combine(p, out, st, true));
   MOE_TRY(mark(5));
   return MOE_OK;
 }
@@ -291,6 +343,18 @@ moe_status moe_layer_forward(const moe_layer* L, const void* x, void* out, int32
                              size_t ws_bytes, moe_stream_t stream) {
   return moe_layer_forward_marked(L, x, out, topk_idx, topk_w, expert_offsets, perm, ws,
                                   ws_bytes, stream, nullptr, 0);
+}
+
+int32_t moe_launches_per_call(const moe_layer* L) {
+  if (validate(L) != MOE_OK) return 0;
+  Plan p{};
+  p.T = L->T;
+  p.E = L->E;
+  p.k = L->k;
+  p.path = L->path;
+  const int route = route_fused_supported(p) ? 1 : (2 + (L->T * L->k <= 1024 ? 1 : 3));
+  const int ffn = use_tc(p) ? 3 : 2;  // (+ gather/schedule) gate/up, down
+  return route + ffn + 1;             // + combine
 }
 
 moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,

@@ -141,66 +141,30 @@ cudaError_t launch_router(const Plan& p, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------------ top-k and gates
-// One warp per token. Lane l holds experts l, l + 32, ...; each of the k rounds takes the
-// warp-wide best (largest value, then lowest index) and retires it.
-__device__ __forceinline__ bool better(float v, int e, float bv, int be) {
-  return v > bv || (v == bv && e < be);
-}
+// One warp per token; the token's keys are staged in shared memory (warp_topk_smem).
+constexpr int kTopkWarps = 4;
 
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
-                                                   int32_t* __restrict__ idx_out,
-                                                   float* __restrict__ w_out, int T, int E,
-                                                   int k) {
-  const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+__global__ void __launch_bounds__(32 * kTopkWarps) topk_kernel(const float* __restrict__ logits,
+                                                               int32_t* __restrict__ idx_out,
+                                                               float* __restrict__ w_out, int T,
+                                                               int E, int k) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int t = blockIdx.x * kTopkWarps + w;
   if (t >= T) return;
-  constexpr int kPer = kMaxE / 32;
-  float v[kPer];
-  const float* row = logits + (size_t)t * E;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = (e < E) ? row[e] : 0.f;
-  }
-  uint32_t taken = 0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i)
-    if (lane + 32 * i >= E) taken |= 1u << i;
-  float sel_v = 0.f;  // lane j keeps the j-th selected value
-  int sel_e = 0;
-  float top = 0.f;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int e = lane + 32 * i;
-      if (!((taken >> i) & 1u) && better(v[i], e, bv, be)) { bv = v[i]; be = e; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == j) { sel_v = bv; sel_e = be; }
-    if (j == 0) top = bv;
-  }
-  const float z = (lane < k) ? expf(sel_v - top) : 0.f;
-  float zs = z;
-  // fixed-order sum over the k selected (lane order = rank order)
-  float total = 0.f;
-  for (int j = 0; j < k; ++j) total += __shfl_sync(0xffffffffu, zs, j);
+  int e;
+  uint32_t key;
+  warp_topk(logits + (size_t)t * E, E, k, lane, &e, &key);
+  const uint32_t top = __shfl_sync(0xffffffffu, key, 0);
+  const float g = warp_topk_gate(key, top, k, lane);
   if (lane < k) {
-    idx_out[(size_t)t * k + lane] = sel_e;
-    w_out[(size_t)t * k + lane] = z / total;
+    idx_out[(size_t)t * k + lane] = e;
+    w_out[(size_t)t * k + lane] = g;
   }
 }
 
 cudaError_t launch_topk(const Plan& p, cudaStream_t st) {
-  const int blocks = (p.T * 32 + 255) / 256;
-  topk_kernel<<<blocks, 256, 0, st>>>(p.logits, p.topk_idx, p.topk_w, p.T, p.E, p.k);
+  const int blocks = (p.T + kTopkWarps - 1) / kTopkWarps;
+  topk_kernel<<<blocks, 32 * kTopkWarps, 0, st>>>(p.logits, p.topk_idx, p.topk_w, p.T, p.E, p.k);
   return cudaGetLastError();
 }
 

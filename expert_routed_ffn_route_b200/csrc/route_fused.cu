@@ -1,0 +1,291 @@
+// Routing and the route plan in one launch, for calls of up to 32 tokens (decode and
+// verify rows), where three separate launches would cost more than the work.
+//
+// Phase 1 (all CTAs): router logits l[t][e] = x_t . Wr_e (+ b_e) in fp32, one warp per
+// expert row, 128-bit loads, every token of the call against the row while it is in
+// registers. Phase 2 (the last CTA to finish phase 1, found with an atomic ticket after a
+// memory fence; nobody waits): per token the stable top-k and the gates, then the
+// expert-major plan and the active-expert list. The ticket is reset for the next call.
+//
+// Rules followed: deterministic stable top-k, ties to the lower expert index
+// (Qwen3.8-Flash-Next-Dual-GPU README, "Independent decode lane"); gates = softmax over the
+// selected logits; plan = counts, exclusive scan, stable scatter (README, "Dedicated
+// prefill lane", step 1).
+#include <cstdlib>
+
+#include "pipeline.cuh"
+
+namespace moe {
+
+#ifdef MOE_TRACE
+__device__ unsigned long long g_ktime[8][4];
+extern "C" __attribute__((visibility("default"))) int moe_ktime_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_ktime, sizeof(g_ktime));
+}
+extern "C" __attribute__((visibility("default"))) int moe_ktime_reset() {
+  unsigned long long h[8][4];
+  for (int i = 0; i < 8; ++i) { h[i][0] = h[i][1] = ~0ull; h[i][2] = h[i][3] = 0; }
+  return (int)cudaMemcpyToSymbol(g_ktime, h, sizeof(h));
+}
+__device__ long long g_rtrace[160][8];
+#define RTRACE(slot) \
+  do { if (threadIdx.x == 0 && blockIdx.x < 160) g_rtrace[blockIdx.x][(slot)] = clock64(); } while (0)
+extern "C" __attribute__((visibility("default"))) int moe_rtrace_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_rtrace, sizeof(g_rtrace));
+}
+#else
+#define RTRACE(slot) do {} while (0)
+#endif
+
+constexpr int kRFWarps = 4;
+constexpr int kRFThreads = 32 * kRFWarps;
+constexpr int kRFMaxT = 32;
+
+__global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t* ticket) {
+  __shared__ int s_last;  // CTA 0: all other CTAs arrived
+  __shared__ int s_idx[kRFMaxT * kMaxK];
+  __shared__ int s_cnt[kMaxE];
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_wsum[kRFWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int T = p.T, E = p.E, d = p.d, k = p.k;
+#ifdef MOE_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 160) {
+    unsigned long long gt;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt));
+    g_rtrace[blockIdx.x][7] = (long long)gt;
+  }
+#endif
+  RTRACE(0);
+  KT_ENTRY(0);
+  pdl_wait();
+  KT_READY(0);
+
+  // ---------------------------------------------------------------- logits
+  // A lane owns 16-byte pieces c = lane + 32 i of the router row (d <= 8192: i < 32); the
+  // row is loaded in batches of 8 pieces, all in flight together, then every token is
+  // applied to the batch while it sits in registers.
+  const int n16 = d / 8;
+  for (int e = blockIdx.x * kRFWarps + warp; e < E; e += gridDim.x * kRFWarps) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(p.router_w + (size_t)e * d);
+    const float b = p.router_bias ? p.router_bias[e] : 0.f;
+    float acc[kRFMaxT];
+#pragma unroll
+    for (int t = 0; t < kRFMaxT; ++t) acc[t] = 0.f;
+    for (int c0 = 0; c0 < n16; c0 += 8 * 32) {
+      uint4 wv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + lane + 32 * i;
+        wv[i] = (c < n16) ? __ldg(wrow + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int t = 0; t < kRFMaxT; ++t) {
+        if (t >= T) break;
+        const uint4* xrow = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
+        uint4 xv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = c0 + lane + 32 * i;
+          xv[i] = (c < n16) ? __ldg(xrow + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+          const uint32_t xx[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[t] = fmaf(__uint_as_float(xx[q] << 16), __uint_as_float(ww[q] << 16), acc[t]);
+            acc[t] = fmaf(__uint_as_float(xx[q] & 0xffff0000u),
+                          __uint_as_float(ww[q] & 0xffff0000u), acc[t]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kRFMaxT; ++t) {
+      if (t >= T) break;
+      float v = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) p.logits[(size_t)t * E + e] = v + b;
+    }
+  }
+
+  // ---------------------------------------------------------------- ticket
+  // CTAs 1.. publish their logits and leave; CTA 0 (always the same one, so the SM that
+  // runs the serial tail below keeps its code in the instruction cache from call to call)
+  // waits, boundedly, until all of them have arrived. All CTAs of this grid are resident
+  // together (gridDim <= E / 4 <= 256, one or two small CTAs per SM).
+  RTRACE(1);
+  __threadfence();
+  __syncthreads();
+  if (blockIdx.x != 0) {
+    if (threadIdx.x == 0) atomicAdd(ticket, 1);
+    if (threadIdx.x == 0) KT_EXIT(0);
+    return;  // an exited CTA counts as having released its dependents
+  }
+  if (threadIdx.x == 0) {
+    const long long t0 = clock64();
+    int seen = 0;
+    while ((seen = *(volatile int*)ticket) < (int)gridDim.x - 1) {
+      if (clock64() - t0 > kWaitCycles) {
+        set_status(p.status, DEV_TIMEOUT);
+        break;
+      }
+    }
+    s_last = (seen >= (int)gridDim.x - 1);
+  }
+  __syncthreads();
+  RTRACE(2);
+  if (!s_last) {  // timed out: leave the outputs untouched; the status word says why
+    if (threadIdx.x == 0) *ticket = 0;
+    pdl_trigger();
+    return;
+  }
+  __threadfence();
+#ifdef MOE_TRACE
+  long long c_fence = clock64();
+#endif
+
+  // ---------------------------------------------------------------- top-k and gates
+  for (int t = warp; t < T; t += kRFWarps) {
+    int e;
+    uint32_t key;
+#ifdef MOE_TRACE
+    long long c_a = clock64();
+#endif
+    warp_topk(p.logits + (size_t)t * E, E, k, lane, &e, &key);
+#ifdef MOE_TRACE
+    if (t == 0 && lane == 0) { g_ktime[7][0] = c_a - c_fence; g_ktime[7][1] = clock64() - c_fence; }
+#endif
+    const uint32_t top = __shfl_sync(0xffffffffu, key, 0);
+    const float g = warp_topk_gate(key, top, k, lane);
+    if (lane < k) {
+      p.topk_idx[(size_t)t * k + lane] = e;
+      p.topk_w[(size_t)t * k + lane] = g;
+      s_idx[t * k + lane] = e;
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  RTRACE(3);
+#ifdef MOE_TRACE
+  if (threadIdx.x == 0) g_ktime[5][1] = clock64() - c_fence;
+#endif
+  // ---------------------------------------------------------------- plan
+  const int n = T * k;
+  if (n <= 32) {
+    // Few assignments: warp 0 ranks them by (expert, index) directly; every thread fills
+    // the offsets of its experts by counting smaller expert ids.
+    __shared__ int s_sorted[32];
+    if (warp == 0) {
+      const int e_me = (lane < n) ? s_idx[lane] : 0x7fffffff;
+      int rank = 0;
+      for (int b = 0; b < n; ++b) {
+        const int eb = __shfl_sync(0xffffffffu, e_me, b);
+        rank += (eb < e_me) || (eb == e_me && b < lane);
+      }
+      if (lane < n) {
+        p.perm[rank] = lane;
+        p.inv[lane] = rank;
+        s_sorted[rank] = e_me;
+      }
+      __syncwarp();
+      const bool first = lane < n && (lane == 0 || s_sorted[lane - 1] != s_sorted[lane]);
+      const unsigned m = __ballot_sync(0xffffffffu, first);
+      if (first) p.active[1 + __popc(m & ((1u << lane) - 1u))] = s_sorted[lane];
+      if (lane == 0) p.active[0] = __popc(m);
+    }
+    for (int e = threadIdx.x; e <= E; e += kRFThreads) {
+      int c = 0;
+      for (int a = 0; a < n; ++a) c += (s_idx[a] < e);
+      p.offsets[e] = c;
+    }
+  } else {
+    for (int e = threadIdx.x; e < E; e += kRFThreads) s_cnt[e] = 0;
+    __syncthreads();
+    for (int a = threadIdx.x; a < n; a += kRFThreads) atomicAdd(&s_cnt[s_idx[a]], 1);
+    __syncthreads();
+    // exclusive scan of s_cnt (each thread owns a contiguous run of experts)
+    const int per = (E + kRFThreads - 1) / kRFThreads;
+    const int e0 = threadIdx.x * per;
+    int local = 0;
+    for (int e = e0; e < min(E, e0 + per); ++e) local += s_cnt[e];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += s_wsum[w];
+    int run = base + incl - local;
+    for (int e = e0; e < min(E, e0 + per); ++e) {
+      s_off[e] = run;
+      p.offsets[e] = run;
+      run += s_cnt[e];
+    }
+    if (threadIdx.x == kRFThreads - 1) {
+      s_off[E] = run;
+      p.offsets[E] = run;
+    }
+    __syncthreads();
+    // active experts in ascending order (warp 0, 32 experts a step)
+    if (warp == 0) {
+      int nact = 0;
+      for (int e0b = 0; e0b < E; e0b += 32) {
+        const int e = e0b + lane;
+        const bool on = (e < E) && s_cnt[e] > 0;
+        const unsigned m = __ballot_sync(0xffffffffu, on);
+        if (on) p.active[1 + nact + __popc(m & ((1u << lane) - 1u))] = e;
+        nact += __popc(m);
+      }
+      if (lane == 0) p.active[0] = nact;
+    }
+    // stable scatter (warp 1; assignments in order, 32 a step)
+    if (warp == 1) {
+      for (int a0 = 0; a0 < n; a0 += 32) {
+        const int a = a0 + lane;
+        const int e = (a < n) ? s_idx[a] : -1;
+        const unsigned m = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(m & ((1u << lane) - 1u));
+        int pos = 0;
+        if (e >= 0) pos = s_off[e] + rank;
+        __syncwarp();
+        if (e >= 0 && (m >> lane) == 1u) s_off[e] += __popc(m);
+        __syncwarp();
+        if (e >= 0) {
+          p.perm[pos] = a;
+          p.inv[a] = pos;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  RTRACE(4);
+#ifdef MOE_TRACE
+  if (threadIdx.x == 0) g_ktime[6][0] = clock64() - c_fence;
+#endif
+  __syncthreads();
+  if (threadIdx.x == 0) *ticket = 0;
+  // The next kernel is released only now: kernels whose CTAs wait early for this one share
+  // the SMs and slow the last CTA down.
+  pdl_trigger();
+  if (threadIdx.x == 0) KT_EXIT(1);
+}
+
+bool route_fused_supported(const Plan& p) { return p.T <= kRFMaxT && p.E <= kMaxE; }
+
+cudaError_t launch_route_fused(const Plan& p, int32_t* ticket, cudaStream_t st) {
+  int blocks = (p.E + kRFWarps - 1) / kRFWarps;
+#ifdef MOE_TRACE
+  if (const char* b = getenv("MOE_RF_BLOCKS")) blocks = atoi(b);
+#endif
+  route_fused_kernel<<<blocks, kRFThreads, 0, st>>>(p, ticket);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

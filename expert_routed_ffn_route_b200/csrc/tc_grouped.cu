@@ -1,0 +1,682 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM), for calls with
+// many rows per expert (prefill slabs): the dense contraction of each expert's rows with its
+// dequantised weights (Qwen3.8-Flash-Next-Dual-GPU README, "Dedicated prefill lane", steps
+// 2-4: grouped W4/W8-A16 tensor-core products over expert-major rows, one fp32 output per
+// assignment; TandemLLM docs, "17 Qwen3.8-Flash-Next", §17.4: rows sorted by expert, one
+// matrix product over each expert's rows).
+//
+// Orientation ("swap AB"): D[n][m] = sum_k W[n][k] X[m][k]; the weights are the M = 128
+// operand (128 rows of one expert matrix), the expert's token rows are N (16..128), K is
+// walked in chunks of 64. D lives in TMEM (lane = weight row, column = token).
+//
+// One persistent CTA per SM, warp roles:
+//   warp 0      TMA producer: raw weight tiles [128 rows x 64 K] (int4/int8/bf16, no
+//               swizzle) and activation tiles [N rows x 64 K] bf16 (128-byte swizzle)
+//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16, bf16 in,
+//               fp32 accumulate
+//   warps 2-5   dequantisers: thread = weight row; W = bf16(q * s) written in the UMMA
+//               K-major 128-byte-swizzled layout, then a proxy fence for the tensor core
+//   warps 6-9   epilogue: tcgen05.ld of their 32 TMEM lanes; gate/up: h = silu(g) * u ->
+//               bf16 rows; down: fp32 rows
+// Rings: raw (TMA -> dequant, activations -> MMA), A (dequant -> MMA), accumulator
+// (MMA -> epilogue, double buffered in TMEM). Every wait is bounded; a timeout sets the
+// status word and every role drains and exits (TMEM is freed by its owner).
+//
+// Work units (slot, n-tile, m-tile) are ordered with the m-tile fastest, and CTAs take
+// them round-robin, so the m-tiles of one weight tile run at the same time on neighbouring
+// SMs and re-read that tile from L2 rather than HBM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "pipeline.cuh"
+
+namespace moe {
+
+constexpr int kTcThreads = 320;
+constexpr int kTcBK = 64;      // K per chunk (one 128-byte swizzle span of bf16)
+constexpr int kTcM = 128;      // weight rows per tile
+constexpr int kTcNMax = 128;   // token rows per tile
+constexpr int kBoxes = 4;      // activation boxes of 16, 32, 64, 128 rows
+
+struct TcMaps {
+  CUtensorMap w[2][2];          // [bank: routed, shared][matrix: gate|down, up]
+  CUtensorMap act[2][kBoxes];   // [source: grouped rows, shared-expert rows][box]
+  int box_rows[2][kBoxes];      // rows per activation box (16 << box, at most the source's)
+};
+
+template <int FMT, bool GATE_UP> struct TcCfg {
+  static constexpr int NM = GATE_UP ? 2 : 1;
+  static constexpr int RAW_ROW = kTcBK * FMT / 8;    // raw bytes of one row per chunk
+  static constexpr int RAW = kTcM * RAW_ROW;         // one raw matrix chunk
+  static constexpr int XB = kTcNMax * kTcBK * 2;     // activation stage bytes
+  static constexpr int AB = kTcM * kTcBK * 2;        // one dequantised matrix chunk
+  static constexpr int NR = GATE_UP ? (FMT == 16 ? 3 : 4) : (FMT == 16 ? 4 : 6);  // raw stages
+  static constexpr int NA = GATE_UP ? 2 : 3;                     // dequantised stages
+  // layout (1024-byte aligned pieces first)
+  static constexpr int X_OFF = 0;
+  static constexpr int A_OFF = X_OFF + NR * XB;
+  static constexpr int R_OFF = A_OFF + NA * NM * AB;
+  static constexpr int BAR_OFF = R_OFF + NR * NM * RAW;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;   // barriers, flags, alignment slack
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// UMMA shared-memory descriptor, K-major, 128-byte swizzle: rows of 128 bytes, groups of
+// 8 rows 1024 bytes apart (SBO), version 1 (sm_100), layout type 2 (128B swizzle).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;                 // LBO (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;       // SBO
+  d |= (uint64_t)1 << 46;                 // version
+  d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(kTcM >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ schedule
+
+struct TcUnit {
+  int slot, e, shared, row0, nrows, ntile, mtile;
+};
+
+__device__ __forceinline__ TcUnit tc_unit(const TcSched& S, int n_slots, int n_tiles, int u) {
+  int lo = 0, hi = n_slots;  // largest s with mt_prefix[s] * n_tiles <= u
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (S.mt_prefix[mid] * n_tiles <= u) lo = mid;
+    else hi = mid;
+  }
+  TcUnit t;
+  t.slot = lo;
+  const int local = u - S.mt_prefix[lo] * n_tiles;
+  const int mts = (S.slot_rows[lo] + kTcNMax - 1) / kTcNMax;
+  t.ntile = local / mts;
+  t.mtile = local % mts;
+  t.e = S.slot_expert[lo];
+  t.shared = (t.e < 0);
+  if (t.shared) t.e = 0;
+  t.row0 = S.slot_row0[lo] + t.mtile * kTcNMax;
+  t.nrows = min(kTcNMax, S.slot_rows[lo] - t.mtile * kTcNMax);
+  return t;
+}
+
+__device__ __forceinline__ int box_index(int nrows) {
+  return nrows <= 16 ? 0 : (nrows <= 32 ? 1 : (nrows <= 64 ? 2 : 3));
+}
+
+// Gathers the routed activation rows into grouped order (xg[r] = x[perm[r] / k]) and, in
+// CTA 0, builds the unit schedule from the plan.
+__global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_t* xg) {
+  pdl_wait();
+  if (blockIdx.x == 0) {
+    __shared__ int s_units[kMaxE + 1];
+    const int n_active = p.active[0];
+    const int n_slots = n_active + (p.has_shared ? 1 : 0);
+    for (int s = threadIdx.x; s < n_slots; s += blockDim.x) {
+      int rows, row0, e;
+      if (s < n_active) {
+        e = p.active[1 + s];
+        row0 = p.offsets[e];
+        rows = p.offsets[e + 1] - row0;
+      } else {
+        e = -1;
+        row0 = 0;
+        rows = p.T;
+      }
+      S.slot_rows[s] = rows;
+      S.slot_row0[s] = row0;
+      S.slot_expert[s] = e;
+      s_units[s] = (rows + kTcNMax - 1) / kTcNMax;  // m-tiles of the slot
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {  // serial prefix over at most E + 1 slots
+      int run = 0;
+      for (int s = 0; s < n_slots; ++s) {
+        S.mt_prefix[s] = run;
+        run += s_units[s];
+      }
+      S.mt_prefix[n_slots] = run;
+    }
+  }
+  {
+    const int n = p.T * p.k;
+    const int chunks = p.d / 8;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < (size_t)n * chunks;
+         i += (size_t)gridDim.x * blockDim.x) {
+      const int r = (int)(i / chunks), c = (int)(i % chunks);
+      const int t = p.perm[r] / p.k;
+      reinterpret_cast<uint4*>(xg + (size_t)r * p.d)[c] =
+          reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d)[c];
+    }
+  }
+  pdl_trigger();
+}
+
+// ------------------------------------------------------------------ dequantisation
+
+// Row r of a raw chunk (64 K values of one weight row) -> 64 bf16 = W * s, stored as the
+// 8 16-byte pieces of row r of a 128-byte-swizzled K-major tile.
+template <int FMT>
+__device__ __forceinline__ void dequant_row(const uint8_t* raw_row, float s, uint8_t* a_tile,
+                                            int r) {
+  uint4 out[8];
+  if constexpr (FMT == 4) {
+    const uint4 q0 = *reinterpret_cast<const uint4*>(raw_row);
+    const uint4 q1 = *reinterpret_cast<const uint4*>(raw_row + 16);
+    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const __nv_bfloat162 s2 = __floats2bfloat162_rn(s, s);
+    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {  // word j = K values 8j .. 8j+7 = output piece j
+      const uint32_t lo = w[j], hi = w[j] >> 4;
+      uint32_t pr[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // byte i of lo holds nibble 2i in its low half, byte i of hi holds nibble 2i+1
+        uint32_t t = __byte_perm(lo, hi, i | ((4 + i) << 8));
+        // keep the low nibble of bytes 0 and 2 (nibbles 2i, 2i+1), flip the sign bit and
+        // place them in the mantissa of 128.0: bf16 values q + 136, exact
+        t = (t & 0x000F000Fu) ^ 0x43084308u;
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&t);
+        v = __hmul2(__hsub2(v, bias), s2);  // q exact, then one rounding of q * s
+        pr[i] = *reinterpret_cast<uint32_t*>(&v);
+      }
+      out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+    }
+  } else if constexpr (FMT == 8) {
+    uint32_t qq[16];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 q = *reinterpret_cast<const uint4*>(raw_row + 16 * v);
+      qq[4 * v] = q.x ^ 0x80808080u;  // u = q + 128 in each byte
+      qq[4 * v + 1] = q.y ^ 0x80808080u;
+      qq[4 * v + 2] = q.z ^ 0x80808080u;
+      qq[4 * v + 3] = q.w ^ 0x80808080u;
+    }
+    // 0x4B000000 | u is the fp32 value 2^23 + u; fma((2^23 + u), s, -(2^23 + 128) s) = q s,
+    // exact (the constant needs 24 significant bits at most), then one rounding to bf16.
+    const float c = -8388736.f * s;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {  // piece j = bytes 8j .. 8j+7 = words 2j, 2j+1
+      uint32_t pr[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t w = qq[2 * j + (i >> 1)];
+        const int b0 = 2 * (i & 1);
+        const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | b0));
+        const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | (b0 + 1)));
+        pr[i] = pack_bf16x2(fmaf(f0, s, c), fmaf(f1, s, c));
+      }
+      out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) out[j] = *reinterpret_cast<const uint4*>(raw_row + 16 * j);
+  }
+  uint8_t* row = a_tile + (size_t)r * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) = out[j];
+}
+
+// ------------------------------------------------------------------ the kernel
+
+template <int FMT, bool GATE_UP>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_grouped_kernel(const __grid_constant__ TcMaps maps, Plan p, TcSched S) {
+  using C = TcCfg<FMT, GATE_UP>;
+  constexpr int NM = C::NM;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* full_raw = bars;                 // [NR]
+  uint64_t* empty_raw = full_raw + C::NR;    // [NR]
+  uint64_t* full_a = empty_raw + C::NR;      // [NA]
+  uint64_t* empty_a = full_a + C::NA;        // [NA]
+  uint64_t* acc_full = empty_a + C::NA;      // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* drain = acc_empty + 2;           // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = GATE_UP ? p.d : p.f;
+  const int N = GATE_UP ? p.f : p.d;
+  const int G = K / kGroup;
+  const int n_tiles = N / kTcM;
+  const int n_chunks = K / kTcBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NR; ++s) {
+      mbar_init(&full_raw[s], 1);
+      mbar_init(&empty_raw[s], 4 + 1);  // 4 dequant warps + the MMA commit
+    }
+    for (int s = 0; s < C::NA; ++s) {
+      mbar_init(&full_a[s], 4);         // 4 dequant warps
+      mbar_init(&empty_a[s], 1);        // MMA commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);       // MMA commit
+      mbar_init(&acc_empty[b], 4);      // 4 epilogue warps
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  pdl_wait();
+  const int n_active = p.active[0];
+  const int n_slots = n_active + (p.has_shared ? 1 : 0);
+  const int total = S.mt_prefix[n_slots] * n_tiles;
+
+  auto fail = [&]() {
+    set_status(p.status, DEV_TIMEOUT);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+        const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
+        const int bx = box_index(t.nrows);
+        const int src = t.shared ? 1 : 0;
+        const int box_rows = maps.box_rows[src][bx];
+        const int wrow = t.e * N + t.ntile * kTcM;
+        const uint32_t bytes = NM * C::RAW + box_rows * kTcBK * 2;
+        for (int c = 0; c < n_chunks; ++c, ++it) {
+          const int s = it % C::NR, use = it / C::NR;
+          if (use > 0 && !mbar_wait(&empty_raw[s], (use - 1) & 1)) {
+            fail();
+            break;
+          }
+          mbar_arrive_expect_tx(&full_raw[s], bytes);
+#pragma unroll
+          for (int mi = 0; mi < NM; ++mi)
+            tma_load_2d(smem + C::R_OFF + (s * NM + mi) * C::RAW, &maps.w[src][mi],
+                        c * C::RAW_ROW, wrow, &full_raw[s]);
+          tma_load_2d(smem + C::X_OFF + s * C::XB, &maps.act[src][bx], c * kTcBK, t.row0,
+                      &full_raw[s]);
+        }
+      }
+      // every issued copy lands before the CTA may exit (consumed ones already have)
+      for (int j = (it > C::NR ? it - C::NR : 0); j < it; ++j)
+        mbar_wait(&full_raw[j % C::NR], (j / C::NR) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, ia = 0, tile = 0;
+      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
+        const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
+        const int n_mma = (t.nrows + 15) & ~15;
+        const uint32_t idesc = umma_idesc_bf16(n_mma);
+        const int b = tile & 1, buse = tile >> 1;
+        if (buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1)) {
+          fail();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem + b * 256;  // gate (or down) accumulator; up at +128
+        bool ok = true;
+        for (int c = 0; c < n_chunks; ++c, ++it, ++ia) {
+          const int s = it % C::NR, a = ia % C::NA;
+          if (!mbar_wait(&full_raw[s], (it / C::NR) & 1) || !mbar_wait(&full_a[a], (ia / C::NA) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xs = smem_u32(smem + C::X_OFF + s * C::XB);
+#pragma unroll
+          for (int kk = 0; kk < kTcBK / 16; ++kk) {
+            const uint64_t bdesc = umma_desc_sw128(xs + kk * 32);
+#pragma unroll
+            for (int mi = 0; mi < NM; ++mi) {
+              const uint32_t as = smem_u32(smem + C::A_OFF + (a * NM + mi) * C::AB);
+              umma_f16(d0 + mi * 128, umma_desc_sw128(as + kk * 32), bdesc, idesc,
+                       (c > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty_raw[s]);
+          umma_commit(&empty_a[a]);
+        }
+        if (!ok) {
+          fail();
+          break;
+        }
+        umma_commit(&acc_full[b]);
+      }
+      // all issued MMAs complete before TMEM and shared memory are released
+      umma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ dequantisers
+    const int r = threadIdx.x - 64;  // weight row in the tile
+    int it = 0, ia = 0;
+    for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+      const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
+      const Bank& bank = t.shared ? p.shared : p.routed;
+      const size_t wrow = (size_t)t.e * N + (size_t)t.ntile * kTcM + r;
+      bool ok = true;
+      for (int c = 0; c < n_chunks; ++c, ++it, ++ia) {
+        const int s = it % C::NR, a = ia % C::NA;
+        float sc[NM];
+#pragma unroll
+        for (int mi = 0; mi < NM; ++mi) {
+          const int which = GATE_UP ? mi : 2;
+          sc[mi] = (FMT == 16) ? 1.f
+                               : bf16_to_f32(__ldg(bank.s[which] + wrow * G + (c * kTcBK) / kGroup));
+        }
+        if (!mbar_wait(&full_raw[s], (it / C::NR) & 1) ||
+            (ia >= C::NA && !mbar_wait(&empty_a[a], ((ia / C::NA) - 1) & 1))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int mi = 0; mi < NM; ++mi) {
+          const uint8_t* raw_row = smem + C::R_OFF + (s * NM + mi) * C::RAW + r * C::RAW_ROW;
+          dequant_row<FMT>(raw_row, sc[mi], smem + C::A_OFF + (a * NM + mi) * C::AB, r);
+        }
+        fence_proxy_async();  // generic-proxy stores -> visible to the tensor core
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&full_a[a]);
+          mbar_arrive(&empty_raw[s]);
+        }
+      }
+      if (!ok) {
+        fail();
+        break;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;     // weight row in the tile
+    int tile = 0;
+    for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
+      const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
+      const int b = tile & 1;
+      if (!mbar_wait(&acc_full[b], (tile >> 1) & 1)) {
+        fail();
+        break;
+      }
+      tc_fence_after();
+      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + b * 256;
+      const int n = t.ntile * kTcM + row;  // output feature
+      for (int m0 = 0; m0 < t.nrows; m0 += 16) {
+        float g[16];
+        tmem_ld16(lane_addr + m0, g);
+        if constexpr (GATE_UP) {
+          float up[16];
+          tmem_ld16(lane_addr + 128 + m0, up);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (m0 + j < t.nrows) {
+              const float h = g[j] / (1.f + expf(-g[j])) * up[j];
+              const size_t hrow = (t.shared ? (size_t)p.T * p.k : 0) + t.row0 + m0 + j;
+              p.h[hrow * p.f + n] = f32_to_bf16_rn(h);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (m0 + j < t.nrows) {
+              float* dst = t.shared ? p.y_shared + (size_t)(t.row0 + m0 + j) * p.d
+                                    : p.y_assign + (size_t)(t.row0 + m0 + j) * p.d;
+              dst[n] = g[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  pdl_trigger();
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [rows][cols] array.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t cols,
+              uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto enc = get_encoder();
+  if (!enc || !base) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t tc_sched_bytes(int E) { return sizeof(int32_t) * (size_t)(4 * (E + 2)); }
+
+TcSched tc_sched_view(void* base, int E) {
+  int32_t* b = static_cast<int32_t*>(base);
+  TcSched s;
+  s.slot_rows = b;
+  s.slot_row0 = b + (E + 2);
+  s.slot_expert = b + 2 * (E + 2);
+  s.mt_prefix = b + 3 * (E + 2);
+  return s;
+}
+
+template <int FMT, bool GATE_UP>
+static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t* xg,
+                                 cudaStream_t st) {
+  using C = TcCfg<FMT, GATE_UP>;
+  const int K = GATE_UP ? p.d : p.f;
+  const int N = GATE_UP ? p.f : p.d;
+  const int wbytes_per_row = K * FMT / 8;  // int4: K/2, int8: K, bf16: 2K
+  const uint32_t box_w = C::RAW_ROW;
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const Bank* banks[2] = {&p.routed, &p.shared};
+  const int nexp[2] = {p.E, p.has_shared ? 1 : 0};
+  for (int b = 0; b < 2; ++b) {
+    if (nexp[b] == 0) continue;
+    for (int mi = 0; mi < C::NM; ++mi) {
+      const int which = GATE_UP ? mi : 2;
+      if (!make_map(&maps.w[b][mi], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, banks[b]->w[which],
+                    wbytes_per_row, (uint64_t)nexp[b] * N, box_w, kTcM,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    }
+  }
+  // activations: grouped rows (gathered x, or h) and the shared expert's rows
+  const uint16_t* act_src[2];
+  uint64_t act_rows[2];
+  if (GATE_UP) {
+    act_src[0] = xg;
+    act_rows[0] = (uint64_t)p.T * p.k;
+    act_src[1] = p.x;
+    act_rows[1] = p.T;
+  } else {
+    act_src[0] = p.h;
+    act_rows[0] = (uint64_t)p.T * p.k;
+    act_src[1] = p.h + (size_t)p.T * p.k * p.f;
+    act_rows[1] = p.T;
+  }
+  for (int s = 0; s < 2; ++s) {
+    if (s == 1 && !p.has_shared) continue;
+    for (int bx = 0; bx < kBoxes; ++bx) {
+      const uint32_t rows = (uint32_t)std::min<uint64_t>(16u << bx, act_rows[s]);
+      maps.box_rows[s][bx] = (int)rows;
+      if (!make_map(&maps.act[s][bx], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act_src[s], K,
+                    act_rows[s], kTcBK, rows, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    }
+  }
+  auto kern = tc_grouped_kernel<FMT, GATE_UP>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int sms = 0;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    int dev = 0;
+    if (attr_err == cudaSuccess) attr_err = cudaGetDevice(&dev);
+    if (attr_err == cudaSuccess)
+      attr_err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, maps, p, S);
+}
+
+template <bool GATE_UP>
+static cudaError_t launch_tc(const Plan& p, const TcSched& S, const uint16_t* xg,
+                             cudaStream_t st) {
+  switch (p.routed.fmt) {
+    case 4: return launch_tc_fmt<4, GATE_UP>(p, S, xg, st);
+    case 8: return launch_tc_fmt<8, GATE_UP>(p, S, xg, st);
+    default: return launch_tc_fmt<16, GATE_UP>(p, S, xg, st);
+  }
+}
+
+bool tc_supported(const Plan& p) {
+  return get_encoder() != nullptr && p.d % kTcM == 0 && p.f % kTcM == 0 &&
+         p.d % kTcBK == 0 && p.f % kTcBK == 0;
+}
+
+cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st) {
+  const long long work = (long long)p.T * p.k * (p.d / 8);
+  const int blocks = (int)std::max(1LL, std::min<long long>(1184, (work + 255) / 256));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_prep_kernel, p, S, xg);
+}
+
+cudaError_t launch_tc_gate_up(const Plan& p, const TcSched& S, const uint16_t* xg,
+                              cudaStream_t st) {
+  return launch_tc<true>(p, S, xg, st);
+}
+cudaError_t launch_tc_down(const Plan& p, const TcSched& S, cudaStream_t st) {
+  return launch_tc<false>(p, S, nullptr, st);
+}
+
+}  // namespace moe

@@ -160,6 +160,10 @@ MOE_API moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, v
                                     int32_t* perm, void* ws, size_t ws_bytes,
                                     moe_stream_t stream, void* const* marks, int32_t n_marks);
 
+/* Number of kernels moe_layer_forward enqueues for this descriptor (0 if L is invalid).
+ * Host-side only; no CUDA call. */
+MOE_API int32_t moe_launches_per_call(const moe_layer* L);
+
 /* Reads the device status word kept in the workspace (synchronises `stream`), writes
  * the code to *code (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE) and clears it. */
 MOE_API moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,

@@ -177,3 +177,34 @@ def test_errors_reported(B, tiny):
     with pytest.raises(B.MoeError) as e:
         B.layer_forward(bad, x, ws)
     assert e.value.status == -1
+
+
+# ------------------------------------------------------------------ tensor-core path
+
+@pytest.mark.parametrize("fmt", ["int4", "int8", "bf16"])
+@pytest.mark.parametrize("shared", [1, 0])
+def test_tc_formats_small(B, fmt, shared):
+    cfg = synth.LayerConfig(f"tc-{fmt}", T=96, d=384, E=12, k=3, f=256, n_shared=shared,
+                            fmt=fmt, seed=11)
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "tc")
+
+
+def test_tc_tiny(B, tiny):
+    L, dl = tiny
+    check_layer(B, dl, L, L.x, "tc")
+
+
+@pytest.mark.parametrize("T", [1, 33])
+def test_tc_ragged_T(B, tiny, T):
+    L, dl = tiny
+    x = synth.make_hidden(L.cfg, L.router_w, L.router_bias, T=T, stream=f"tcragged{T}")
+    check_layer(B, dl, L, x, "tc")
+
+
+def test_tc_many_m_tiles(B):
+    """One expert gets several 128-row m-tiles (skewed routing), ragged last tile."""
+    cfg = synth.LayerConfig("tc-hot", T=700, d=256, E=8, k=2, f=256, fmt="int8", zipf_s=3.0,
+                            seed=13)
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "tc", sample=[0, 1, 350, 699])
