@@ -12,7 +12,7 @@
 namespace moe {
 
 // Status word kept at the start of the workspace (device side).
-enum : int32_t { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BOUNDS = 2 };
+enum : int32_t { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BOUNDS = 2, DEV_RANGE = 3 };
 
 constexpr int kGroup = 128;      // quantisation group along K
 constexpr int kMaxE = 1024;      // experts a layer
@@ -155,7 +155,8 @@ struct Plan {
   float* y_shared;     // [T*d]
   int32_t* status;
   int32_t* ticket;     // zero between calls; the fused routing kernel's completion counter
-  uint16_t* xg;        // tensor-core path: x rows gathered into grouped order [T*k][d]
+  uint16_t* xg;        // tensor-core path: fp16 x rows in grouped order, then the shared
+                       // expert's rows [(T*k + T)][d]
   int32_t* tc_sched;   // tensor-core path: per-slot schedule (TcSched view)
   int path;            // moe_path
 };

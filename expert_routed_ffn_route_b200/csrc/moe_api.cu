@@ -72,7 +72,7 @@ WsLayout layout(const moe_layer* L) {
   w.h = take((n + T) * f * sizeof(uint16_t));
   w.y_assign = take(n * d * sizeof(float));
   w.y_shared = take(T * d * sizeof(float));
-  w.xg = take(n * d * sizeof(uint16_t));
+  w.xg = take((n + T) * d * sizeof(uint16_t));
   w.tc_sched = take(tc_sched_bytes(L->E));
   w.total = o;
   return w;
@@ -167,7 +167,9 @@ bool use_tc(const Plan& p) {
 
 moe_status run_ffn(const Plan& p, cudaStream_t st, void* const* marks, int n_marks) {
   if (use_tc(p)) {
-    if (!tc_supported(p)) return MOE_ERR_UNSUPPORTED;
+    if (!tc_supported(p) || !scales_aligned16(p.routed) ||
+        (p.has_shared && !scales_aligned16(p.shared)))
+      return MOE_ERR_UNSUPPORTED;
     const TcSched S = tc_sched_view(p.tc_sched, p.E);
     MOE_TRY(launch_tc_prep(p, S, p.xg, st));
     MOE_TRY(launch_tc_gate_up(p, S, p.xg, st));

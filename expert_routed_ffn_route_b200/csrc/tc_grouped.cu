@@ -12,14 +12,20 @@
 // One persistent CTA per SM, warp roles:
 //   warp 0      TMA producer: raw weight tiles [128 rows x 64 K] (int4/int8/bf16, no
 //               swizzle) and activation tiles [N rows x 64 K] bf16 (128-byte swizzle)
-//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16, bf16 in,
-//               fp32 accumulate
-//   warps 2-5   dequantisers: thread = weight row; W = bf16(q * s) written in the UMMA
-//               K-major 128-byte-swizzled layout, then a proxy fence for the tensor core
-//   warps 6-9   epilogue: tcgen05.ld of their 32 TMEM lanes; gate/up: h = silu(g) * u ->
-//               bf16 rows; down: fp32 rows
-// Rings: raw (TMA -> dequant, activations -> MMA), A (dequant -> MMA), accumulator
-// (MMA -> epilogue, double buffered in TMEM). Every wait is bounded; a timeout sets the
+//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16, fp32
+//               accumulate; for gate/up warp 14 issues the up-projection MMAs in parallel
+//               (separate accumulator), which halves the instructions one thread issues
+//   warps 2-9   dequantisers: two threads per weight row, W = fp16(q * s) written straight
+//               from registers into TMEM (tcgen05.st), where the MMA reads its A operand;
+//               shared memory then carries only the raw weights and the activations
+//   warps 10-13 epilogue: tcgen05.ld of their 32 TMEM lanes; gate/up: h = silu(g) * u ->
+//               fp16 rows; down: fp32 rows
+// Operands are fp16 (kind::f16, fp32 accumulate): the activations (bf16 inputs) convert to
+// fp16 exactly in fp16's range, and q * s rounds once with an 11-bit significand, eight
+// times finer than bf16. Activations and h outside fp16's range set a device status flag.
+// Rings: weights (TMA -> dequant), activations (TMA -> MMA), A (dequant -> MMA, in TMEM),
+// accumulator (MMA -> epilogue, double buffered in TMEM). TMEM columns: accumulators
+// [0, 256) (buffer b: gate at 128 b, up at 128 b + 64), A stages [256, 512). Every wait is bounded; a timeout sets the
 // status word and every role drains and exits (TMEM is freed by its owner).
 //
 // Work units (slot, n-tile, m-tile) are ordered with the m-tile fastest, and CTAs take
@@ -31,15 +37,36 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda_fp16.h>
+
 #include "pipeline.cuh"
 
 namespace moe {
 
-constexpr int kTcThreads = 320;
+#ifdef MOE_TRACE
+__device__ long long g_tct[2][4][16][2];  // [kernel][role][unit][start/end], CTA 0
+#define TCT(role, ui, se) \
+  do { if (blockIdx.x == 0 && (ui) < 16) g_tct[GATE_UP ? 0 : 1][role][ui][se] = clock64(); } while (0)
+__device__ long long g_tcc[2][48][6];  // [kernel][chunk of unit 0][event], CTA 0
+#define TCC(c, ev) \
+  do { if (blockIdx.x == 0 && (c) < 48) g_tcc[GATE_UP ? 0 : 1][c][ev] = clock64(); } while (0)
+extern "C" __attribute__((visibility("default"))) int moe_tcc_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_tcc, sizeof(g_tcc));
+}
+extern "C" __attribute__((visibility("default"))) int moe_tct_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_tct, sizeof(g_tct));
+}
+#else
+#define TCT(role, ui, se) do {} while (0)
+#define TCC(c, ev) do {} while (0)
+#endif
+
+constexpr int kTcThreads = 480;  // 15 warps
+constexpr int kDqWarps = 8;       // dequantisers (two threads per weight row)
 constexpr int kTcBK = 64;      // K per chunk (one 128-byte swizzle span of bf16)
 constexpr int kTcM = 128;      // weight rows per tile
-constexpr int kTcNMax = 128;   // token rows per tile
-constexpr int kBoxes = 4;      // activation boxes of 16, 32, 64, 128 rows
+constexpr int kTcNMax = 64;    // token rows per tile
+constexpr int kBoxes = 3;      // activation boxes of 16, 32, 64 rows
 
 struct TcMaps {
   CUtensorMap w[2][2];          // [bank: routed, shared][matrix: gate|down, up]
@@ -52,17 +79,41 @@ template <int FMT, bool GATE_UP> struct TcCfg {
   static constexpr int RAW_ROW = kTcBK * FMT / 8;    // raw bytes of one row per chunk
   static constexpr int RAW = kTcM * RAW_ROW;         // one raw matrix chunk
   static constexpr int XB = kTcNMax * kTcBK * 2;     // activation stage bytes
-  static constexpr int AB = kTcM * kTcBK * 2;        // one dequantised matrix chunk
-  static constexpr int NR = GATE_UP ? (FMT == 16 ? 3 : 4) : (FMT == 16 ? 4 : 6);  // raw stages
-  static constexpr int NA = GATE_UP ? 2 : 3;                     // dequantised stages
+  // Ring depths: the weight ring is deep (HBM latency) and is released by the dequantisers
+  // as soon as they have read it; the activation ring (mostly L2 hits) by the tensor core.
+  static constexpr int WB = NM * RAW;                // weight stage bytes
+  static constexpr int W_BUDGET = (GATE_UP ? 128 : 96) * 1024;
+  static constexpr int NW = W_BUDGET / WB > 16 ? 16 : W_BUDGET / WB;
+  static constexpr int NX = 6;
+  static constexpr int A_COLS = NM * (kTcBK / 2);    // TMEM columns of one A stage
+  static constexpr int NA = GATE_UP ? 4 : 6;         // A stages in TMEM
+  static constexpr int A_COL0 = 256;
+  static_assert(A_COL0 + NA * A_COLS <= 512, "TMEM budget");
   // layout (1024-byte aligned pieces first)
   static constexpr int X_OFF = 0;
-  static constexpr int A_OFF = X_OFF + NR * XB;
-  static constexpr int R_OFF = A_OFF + NA * NM * AB;
-  static constexpr int BAR_OFF = R_OFF + NR * NM * RAW;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;   // barriers, flags, alignment slack
-  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static constexpr int R_OFF = X_OFF + NX * XB;
+  static constexpr int S_OFF = R_OFF + NW * WB;      // then: unit scales, schedule, barriers
+  static_assert(S_OFF + 32 * 1024 <= 227 * 1024, "shared memory budget");
 };
+
+// Runtime part of the shared-memory layout: per-unit scale blocks (double buffered) of
+// kTcM rows x K/128 bf16 per matrix, the schedule cache and the barriers.
+struct TcSmem {
+  int sb;                       // bytes of one matrix's scale block
+  int sched_off, bar_off, total;
+};
+
+template <int FMT, bool GATE_UP>
+__host__ __device__ inline TcSmem tc_smem(int K, int E) {
+  using C = TcCfg<FMT, GATE_UP>;
+  TcSmem m;
+  m.sb = (FMT == 16) ? 0 : kTcM * (K / kGroup) * 2;
+  m.sched_off = C::S_OFF + 2 * C::NM * m.sb;
+  m.bar_off = m.sched_off + 4 * (E + 2) * (int)sizeof(int32_t);
+  m.bar_off = (m.bar_off + 15) & ~15;
+  m.total = m.bar_off + 512 + 1024;  // barriers and flags, 1024 bytes of alignment slack
+  return m;
+}
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -104,6 +155,31 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// A operand from TMEM (row = lane, K packed two fp16 per 32-bit column), B from shared memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane <- registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -138,10 +214,9 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = n.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(kTcM >> 4) << 24);
+// Instruction descriptor: D fp32, A and B fp16, both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTcM >> 4) << 24);
 }
 
 // ------------------------------------------------------------------ schedule
@@ -150,6 +225,7 @@ struct TcUnit {
   int slot, e, shared, row0, nrows, ntile, mtile;
 };
 
+// S points at the CTA's shared-memory copy of the schedule.
 __device__ __forceinline__ TcUnit tc_unit(const TcSched& S, int n_slots, int n_tiles, int u) {
   int lo = 0, hi = n_slots;  // largest s with mt_prefix[s] * n_tiles <= u
   while (hi - lo > 1) {
@@ -175,8 +251,8 @@ __device__ __forceinline__ int box_index(int nrows) {
   return nrows <= 16 ? 0 : (nrows <= 32 ? 1 : (nrows <= 64 ? 2 : 3));
 }
 
-// Gathers the routed activation rows into grouped order (xg[r] = x[perm[r] / k]) and, in
-// CTA 0, builds the unit schedule from the plan.
+// Gathers the activation rows in fp16 (xg[r] = x[perm[r] / k] for the T*k grouped rows, then
+// xg[T*k + t] = x[t] for the shared expert) and, in CTA 0, builds the unit schedule.
 __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_t* xg) {
   pdl_wait();
   if (blockIdx.x == 0) {
@@ -211,64 +287,71 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
   }
   {
     const int n = p.T * p.k;
+    const int rows = n + (p.has_shared ? p.T : 0);
     const int chunks = p.d / 8;
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < (size_t)n * chunks;
+    bool range_ok = true;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < (size_t)rows * chunks;
          i += (size_t)gridDim.x * blockDim.x) {
       const int r = (int)(i / chunks), c = (int)(i % chunks);
-      const int t = p.perm[r] / p.k;
-      reinterpret_cast<uint4*>(xg + (size_t)r * p.d)[c] =
-          reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d)[c];
+      const int t = (r < n) ? p.perm[r] / p.k : r - n;
+      const uint4 v = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d)[c];
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = __uint_as_float(vv[q] << 16), b = __uint_as_float(vv[q] & 0xffff0000u);
+        range_ok &= (fabsf(a) <= 65504.f) && (fabsf(b) <= 65504.f);
+        __half2 h = __floats2half2_rn(a, b);
+        o[q] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(xg + (size_t)r * p.d)[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    if (!range_ok) set_status(p.status, DEV_RANGE);
   }
   pdl_trigger();
 }
 
 // ------------------------------------------------------------------ dequantisation
 
-// Row r of a raw chunk (64 K values of one weight row) -> 64 bf16 = W * s, stored as the
-// 8 16-byte pieces of row r of a 128-byte-swizzled K-major tile.
+// Half `half` (K values 32*half .. 32*half+31) of a raw chunk row (64 K values of one
+// weight row) -> 32 fp16 = W * s in K order, two per register.
 template <int FMT>
-__device__ __forceinline__ void dequant_row(const uint8_t* raw_row, float s, uint8_t* a_tile,
-                                            int r) {
-  uint4 out[8];
+__device__ __forceinline__ void dequant_half_row(const uint8_t* raw_row, float s, int half,
+                                                 uint32_t (&outr)[16]) {
+  uint4 out[4];
   if constexpr (FMT == 4) {
-    const uint4 q0 = *reinterpret_cast<const uint4*>(raw_row);
-    const uint4 q1 = *reinterpret_cast<const uint4*>(raw_row + 16);
-    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    const __nv_bfloat162 s2 = __floats2bfloat162_rn(s, s);
-    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.f, 136.f);
+    const uint4 q = *reinterpret_cast<const uint4*>(raw_row + 16 * half);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    const __half2 s2 = __float2half2_rn(s);
+    const __half2 bias = __float2half2_rn(1032.f);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {  // word j = K values 8j .. 8j+7 = output piece j
+    for (int j = 0; j < 4; ++j) {  // word j = K values 8j .. 8j+7 of this half
       const uint32_t lo = w[j], hi = w[j] >> 4;
       uint32_t pr[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        // byte i of lo holds nibble 2i in its low half, byte i of hi holds nibble 2i+1
+        // byte i of lo holds nibble 2i in its low half, byte i of hi holds nibble 2i+1;
+        // keep those two nibbles, flip their sign bit and place them in the mantissa of
+        // 1024.0: fp16 values 1024 + (n ^ 8) = q + 1032, exact
         uint32_t t = __byte_perm(lo, hi, i | ((4 + i) << 8));
-        // keep the low nibble of bytes 0 and 2 (nibbles 2i, 2i+1), flip the sign bit and
-        // place them in the mantissa of 128.0: bf16 values q + 136, exact
-        t = (t & 0x000F000Fu) ^ 0x43084308u;
-        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&t);
+        t = (t & 0x000F000Fu) ^ 0x64086408u;
+        __half2 v = *reinterpret_cast<__half2*>(&t);
         v = __hmul2(__hsub2(v, bias), s2);  // q exact, then one rounding of q * s
         pr[i] = *reinterpret_cast<uint32_t*>(&v);
       }
       out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
     }
   } else if constexpr (FMT == 8) {
-    uint32_t qq[16];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 q = *reinterpret_cast<const uint4*>(raw_row + 16 * v);
-      qq[4 * v] = q.x ^ 0x80808080u;  // u = q + 128 in each byte
-      qq[4 * v + 1] = q.y ^ 0x80808080u;
-      qq[4 * v + 2] = q.z ^ 0x80808080u;
-      qq[4 * v + 3] = q.w ^ 0x80808080u;
-    }
+    const uint4 q0 = *reinterpret_cast<const uint4*>(raw_row + 32 * half);
+    const uint4 q1 = *reinterpret_cast<const uint4*>(raw_row + 32 * half + 16);
+    const uint32_t qq[8] = {q0.x ^ 0x80808080u, q0.y ^ 0x80808080u, q0.z ^ 0x80808080u,
+                            q0.w ^ 0x80808080u, q1.x ^ 0x80808080u, q1.y ^ 0x80808080u,
+                            q1.z ^ 0x80808080u, q1.w ^ 0x80808080u};  // u = q + 128 per byte
     // 0x4B000000 | u is the fp32 value 2^23 + u; fma((2^23 + u), s, -(2^23 + 128) s) = q s,
-    // exact (the constant needs 24 significant bits at most), then one rounding to bf16.
+    // exact (the constant needs 24 significant bits at most), then one rounding to fp16.
     const float c = -8388736.f * s;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {  // piece j = bytes 8j .. 8j+7 = words 2j, 2j+1
+    for (int j = 0; j < 4; ++j) {  // piece j = bytes 8j .. 8j+7 = words 2j, 2j+1
       uint32_t pr[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -276,17 +359,33 @@ __device__ __forceinline__ void dequant_row(const uint8_t* raw_row, float s, uin
         const int b0 = 2 * (i & 1);
         const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | b0));
         const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | (b0 + 1)));
-        pr[i] = pack_bf16x2(fmaf(f0, s, c), fmaf(f1, s, c));
+        __half2 h = __floats2half2_rn(fmaf(f0, s, c), fmaf(f1, s, c));
+        pr[i] = *reinterpret_cast<uint32_t*>(&h);
       }
       out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) out[j] = *reinterpret_cast<const uint4*>(raw_row + 16 * j);
-  }
-  uint8_t* row = a_tile + (size_t)r * 128;
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = *reinterpret_cast<const uint4*>(raw_row + 64 * half + 16 * j);
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t pr[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) << 4)) = out[j];
+      for (int i = 0; i < 4; ++i) {
+        __half2 h = __floats2half2_rn(__uint_as_float(vv[i] << 16),
+                                      __uint_as_float(vv[i] & 0xffff0000u));
+        pr[i] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    outr[4 * j] = out[j].x;
+    outr[4 * j + 1] = out[j].y;
+    outr[4 * j + 2] = out[j].z;
+    outr[4 * j + 3] = out[j].w;
+  }
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -300,14 +399,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* full_raw = bars;                 // [NR]
-  uint64_t* empty_raw = full_raw + C::NR;    // [NR]
-  uint64_t* full_a = empty_raw + C::NR;      // [NA]
+  const TcSmem SL = tc_smem<FMT, GATE_UP>(GATE_UP ? p.d : p.f, p.E);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bar_off);
+  uint64_t* full_w = bars;                   // [NW]
+  uint64_t* empty_w = full_w + C::NW;        // [NW]
+  uint64_t* full_x = empty_w + C::NW;        // [NX]
+  uint64_t* empty_x = full_x + C::NX;        // [NX]
+  uint64_t* full_a = empty_x + C::NX;        // [NA]
   uint64_t* empty_a = full_a + C::NA;        // [NA]
   uint64_t* acc_full = empty_a + C::NA;      // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
-  uint64_t* drain = acc_empty + 2;           // [1]
+  uint64_t* scale_full = acc_empty + 2;      // [2] one per unit parity
+  uint64_t* scale_empty = scale_full + 2;    // [2]
+  uint64_t* drain = scale_empty + 2;         // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -319,19 +423,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int n_chunks = K / kTcBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NR; ++s) {
-      mbar_init(&full_raw[s], 1);
-      mbar_init(&empty_raw[s], 4 + 1);  // 4 dequant warps + the MMA commit
+    for (int s = 0; s < C::NW; ++s) {
+      mbar_init(&full_w[s], 1);
+      mbar_init(&empty_w[s], kDqWarps);  // dequant warps
+    }
+    for (int s = 0; s < C::NX; ++s) {
+      mbar_init(&full_x[s], 1);
+      mbar_init(&empty_x[s], NM);        // one MMA commit per issuer
     }
     for (int s = 0; s < C::NA; ++s) {
-      mbar_init(&full_a[s], 4);         // 4 dequant warps
-      mbar_init(&empty_a[s], 1);        // MMA commit
+      mbar_init(&full_a[s], kDqWarps);  // dequant warps
+      mbar_init(&empty_a[s], NM);       // one MMA commit per issuer
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);       // MMA commit
+      mbar_init(&acc_full[b], NM);      // one MMA commit per issuer
       mbar_init(&acc_empty[b], 4);      // 4 epilogue warps
     }
-    mbar_init(drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&scale_full[b], 1);
+      mbar_init(&scale_empty[b], kDqWarps);
+    }
+    mbar_init(drain, NM);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -344,7 +456,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   pdl_wait();
   const int n_active = p.active[0];
   const int n_slots = n_active + (p.has_shared ? 1 : 0);
-  const int total = S.mt_prefix[n_slots] * n_tiles;
+  // schedule -> shared memory (every role looks units up many times)
+  TcSched Ss;
+  {
+    int32_t* sc = reinterpret_cast<int32_t*>(smem + SL.sched_off);
+    Ss.slot_rows = sc;
+    Ss.slot_row0 = sc + (p.E + 2);
+    Ss.slot_expert = sc + 2 * (p.E + 2);
+    Ss.mt_prefix = sc + 3 * (p.E + 2);
+    for (int i = threadIdx.x; i <= n_slots; i += blockDim.x) {
+      Ss.mt_prefix[i] = S.mt_prefix[i];
+      if (i < n_slots) {
+        Ss.slot_rows[i] = S.slot_rows[i];
+        Ss.slot_row0[i] = S.slot_row0[i];
+        Ss.slot_expert[i] = S.slot_expert[i];
+      }
+    }
+  }
+  __syncthreads();
+  const int total = Ss.mt_prefix[n_slots] * n_tiles;
 
   auto fail = [&]() {
     set_status(p.status, DEV_TIMEOUT);
@@ -354,147 +484,190 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int it = 0;
-      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
-        const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
+      int it = 0, ui = 0;
+      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++ui) {
+        const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
         const int bx = box_index(t.nrows);
         const int src = t.shared ? 1 : 0;
         const int box_rows = maps.box_rows[src][bx];
         const int wrow = t.e * N + t.ntile * kTcM;
-        const uint32_t bytes = NM * C::RAW + box_rows * kTcBK * 2;
-        for (int c = 0; c < n_chunks; ++c, ++it) {
-          const int s = it % C::NR, use = it / C::NR;
-          if (use > 0 && !mbar_wait(&empty_raw[s], (use - 1) & 1)) {
+        TCT(0, ui, 0);
+        if constexpr (FMT != 16) {
+          // the unit's group scales: kTcM consecutive rows, one contiguous block per matrix
+          const int sbuf = ui & 1;
+          if (ui >= 2 && !mbar_wait(&scale_empty[sbuf], ((ui >> 1) - 1) & 1)) {
             fail();
             break;
           }
-          mbar_arrive_expect_tx(&full_raw[s], bytes);
+          mbar_arrive_expect_tx(&scale_full[sbuf], (uint32_t)(NM * SL.sb));
+          const Bank& bank = t.shared ? p.shared : p.routed;
+#pragma unroll
+          for (int mi = 0; mi < NM; ++mi) {
+            const int which = GATE_UP ? mi : 2;
+            bulk_g2s(smem + C::S_OFF + (sbuf * NM + mi) * SL.sb, bank.s[which] + (size_t)wrow * G,
+                     (uint32_t)SL.sb, &scale_full[sbuf]);
+          }
+        }
+        for (int c = 0; c < n_chunks; ++c, ++it) {
+          const int sw = it % C::NW, uw = it / C::NW;
+          const int sx = it % C::NX, ux = it / C::NX;
+          if ((uw > 0 && !mbar_wait(&empty_w[sw], (uw - 1) & 1)) ||
+              (ux > 0 && !mbar_wait(&empty_x[sx], (ux - 1) & 1))) {
+            fail();
+            break;
+          }
+          mbar_arrive_expect_tx(&full_w[sw], (uint32_t)C::WB);
 #pragma unroll
           for (int mi = 0; mi < NM; ++mi)
-            tma_load_2d(smem + C::R_OFF + (s * NM + mi) * C::RAW, &maps.w[src][mi],
-                        c * C::RAW_ROW, wrow, &full_raw[s]);
-          tma_load_2d(smem + C::X_OFF + s * C::XB, &maps.act[src][bx], c * kTcBK, t.row0,
-                      &full_raw[s]);
+            tma_load_2d(smem + C::R_OFF + sw * C::WB + mi * C::RAW, &maps.w[src][mi],
+                        c * C::RAW_ROW, wrow, &full_w[sw]);
+          mbar_arrive_expect_tx(&full_x[sx], (uint32_t)(box_rows * kTcBK * 2));
+          tma_load_2d(smem + C::X_OFF + sx * C::XB, &maps.act[src][bx], c * kTcBK, t.row0,
+                      &full_x[sx]);
         }
+        TCT(0, ui, 1);
       }
       // every issued copy lands before the CTA may exit (consumed ones already have)
-      for (int j = (it > C::NR ? it - C::NR : 0); j < it; ++j)
-        mbar_wait(&full_raw[j % C::NR], (j / C::NR) & 1);
+      for (int j = (it > C::NW ? it - C::NW : 0); j < it; ++j)
+        mbar_wait(&full_w[j % C::NW], (j / C::NW) & 1);
+      for (int j = (it > C::NX ? it - C::NX : 0); j < it; ++j)
+        mbar_wait(&full_x[j % C::NX], (j / C::NX) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp == 1 || warp == 14) {
+    // ------------------------------------------------------------ MMA issuers
+    const int mi = (warp == 1) ? 0 : 1;  // matrix this thread issues
+    if (lane == 0 && mi < NM) {
       int it = 0, ia = 0, tile = 0;
       for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
-        const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
+        const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
         const int n_mma = (t.nrows + 15) & ~15;
-        const uint32_t idesc = umma_idesc_bf16(n_mma);
+        const uint32_t idesc = umma_idesc_f16(n_mma);
         const int b = tile & 1, buse = tile >> 1;
         if (buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1)) {
           fail();
           break;
         }
         tc_fence_after();
-        const uint32_t d0 = tmem + b * 256;  // gate (or down) accumulator; up at +128
+        TCT(1, tile, 0);
+        const uint32_t d0 = tmem + b * 128;  // gate (or down) accumulator; up at +64
         bool ok = true;
         for (int c = 0; c < n_chunks; ++c, ++it, ++ia) {
-          const int s = it % C::NR, a = ia % C::NA;
-          if (!mbar_wait(&full_raw[s], (it / C::NR) & 1) || !mbar_wait(&full_a[a], (ia / C::NA) & 1)) {
+          const int sx = it % C::NX, a = ia % C::NA;
+          const bool okx = mbar_wait(&full_x[sx], (it / C::NX) & 1);
+          TCC(it, 0);
+          const bool oka = okx && mbar_wait(&full_a[a], (ia / C::NA) & 1);
+          TCC(it, 1);
+          if (!oka) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t xs = smem_u32(smem + C::X_OFF + s * C::XB);
+          const uint32_t xs = smem_u32(smem + C::X_OFF + sx * C::XB);
 #pragma unroll
           for (int kk = 0; kk < kTcBK / 16; ++kk) {
             const uint64_t bdesc = umma_desc_sw128(xs + kk * 32);
-#pragma unroll
-            for (int mi = 0; mi < NM; ++mi) {
-              const uint32_t as = smem_u32(smem + C::A_OFF + (a * NM + mi) * C::AB);
-              umma_f16(d0 + mi * 128, umma_desc_sw128(as + kk * 32), bdesc, idesc,
-                       (c > 0 || kk > 0) ? 1u : 0u);
-            }
+            const uint32_t at = tmem + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2) + kk * 8;
+            umma_f16_ts(d0 + mi * kTcNMax, at, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&empty_raw[s]);
+          umma_commit(&empty_x[sx]);
           umma_commit(&empty_a[a]);
+          TCC(it, 2);
         }
         if (!ok) {
           fail();
           break;
         }
         umma_commit(&acc_full[b]);
+        TCT(1, tile, 1);
       }
       // all issued MMAs complete before TMEM and shared memory are released
       umma_commit(drain);
       mbar_wait(drain, 0);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kDqWarps) {
     // ------------------------------------------------------------ dequantisers
-    const int r = threadIdx.x - 64;  // weight row in the tile
-    int it = 0, ia = 0;
-    for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
-      const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
-      const Bank& bank = t.shared ? p.shared : p.routed;
-      const size_t wrow = (size_t)t.e * N + (size_t)t.ntile * kTcM + r;
+    // TMEM lanes a warp may write are 32 * (warp % 4) .. +31: rows follow the warp
+    const int r = 32 * (warp & 3) + lane;            // weight row in the tile
+    const int half = (warp - 2) >> 2;                // which 32 K values of the chunk
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    int it = 0, ia = 0, ui = 0;
+    for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++ui) {
+      const int sbuf = ui & 1;
       bool ok = true;
-      for (int c = 0; c < n_chunks; ++c, ++it, ++ia) {
-        const int s = it % C::NR, a = ia % C::NA;
+      if (threadIdx.x == 64) TCT(2, ui, 0);
+      if constexpr (FMT != 16) ok = mbar_wait(&scale_full[sbuf], (ui >> 1) & 1);
+      const uint16_t* sblk = reinterpret_cast<const uint16_t*>(smem + C::S_OFF + sbuf * NM * SL.sb);
+      for (int c = 0; c < n_chunks && ok; ++c, ++it, ++ia) {
+        const int sw = it % C::NW, a = ia % C::NA;
         float sc[NM];
 #pragma unroll
-        for (int mi = 0; mi < NM; ++mi) {
-          const int which = GATE_UP ? mi : 2;
+        for (int mi = 0; mi < NM; ++mi)
           sc[mi] = (FMT == 16) ? 1.f
-                               : bf16_to_f32(__ldg(bank.s[which] + wrow * G + (c * kTcBK) / kGroup));
-        }
-        if (!mbar_wait(&full_raw[s], (it / C::NR) & 1) ||
-            (ia >= C::NA && !mbar_wait(&empty_a[a], ((ia / C::NA) - 1) & 1))) {
+                               : bf16_to_f32(sblk[mi * (SL.sb / 2) + r * G + (c * kTcBK) / kGroup]);
+        const bool okw = mbar_wait(&full_w[sw], (it / C::NW) & 1);
+        if (threadIdx.x == 64) TCC(it, 3);
+        const bool oka = okw && (ia < C::NA || mbar_wait(&empty_a[a], ((ia / C::NA) - 1) & 1));
+        if (threadIdx.x == 64) TCC(it, 4);
+        if (!oka) {
           ok = false;
           break;
         }
 #pragma unroll
         for (int mi = 0; mi < NM; ++mi) {
-          const uint8_t* raw_row = smem + C::R_OFF + (s * NM + mi) * C::RAW + r * C::RAW_ROW;
-          dequant_row<FMT>(raw_row, sc[mi], smem + C::A_OFF + (a * NM + mi) * C::AB, r);
+          const uint8_t* raw_row = smem + C::R_OFF + sw * C::WB + mi * C::RAW + r * C::RAW_ROW;
+          uint32_t regs[16];
+          dequant_half_row<FMT>(raw_row, sc[mi], half, regs);
+          tmem_st16(lane_base + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2) + 16 * half, regs);
         }
-        fence_proxy_async();  // generic-proxy stores -> visible to the tensor core
+        tmem_st_wait();
+        tc_fence_before();  // the stores are complete before the arrive below
         __syncwarp();
+        if (threadIdx.x == 64) TCC(it, 5);
         if (lane == 0) {
           mbar_arrive(&full_a[a]);
-          mbar_arrive(&empty_raw[s]);
+          mbar_arrive(&empty_w[sw]);
         }
       }
       if (!ok) {
         fail();
         break;
       }
+      if constexpr (FMT != 16) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&scale_empty[sbuf]);
+      }
+      if (threadIdx.x == 64) TCT(2, ui, 1);
     }
-  } else {
+  } else if (warp < 14) {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31 (warps 10..13)
     const int row = quarter * 32 + lane;     // weight row in the tile
     int tile = 0;
     for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
-      const TcUnit t = tc_unit(S, n_slots, n_tiles, u);
+      const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
       const int b = tile & 1;
       if (!mbar_wait(&acc_full[b], (tile >> 1) & 1)) {
         fail();
         break;
       }
       tc_fence_after();
-      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + b * 256;
+      if (threadIdx.x == 320) TCT(3, tile, 0);
+      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + b * 128;
       const int n = t.ntile * kTcM + row;  // output feature
       for (int m0 = 0; m0 < t.nrows; m0 += 16) {
         float g[16];
         tmem_ld16(lane_addr + m0, g);
         if constexpr (GATE_UP) {
           float up[16];
-          tmem_ld16(lane_addr + 128 + m0, up);
+          tmem_ld16(lane_addr + kTcNMax + m0, up);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (m0 + j < t.nrows) {
               const float h = g[j] / (1.f + expf(-g[j])) * up[j];
               const size_t hrow = (t.shared ? (size_t)p.T * p.k : 0) + t.row0 + m0 + j;
-              p.h[hrow * p.f + n] = f32_to_bf16_rn(h);
+              if (!(fabsf(h) <= 65504.f)) set_status(p.status, DEV_RANGE);
+              const __half hh = __float2half_rn(h);
+              p.h[hrow * p.f + n] = *reinterpret_cast<const uint16_t*>(&hh);
             }
           }
         } else {
@@ -511,6 +684,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
+      if (threadIdx.x == 320) TCT(3, tile, 1);
     }
   }
 
@@ -598,7 +772,7 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
   if (GATE_UP) {
     act_src[0] = xg;
     act_rows[0] = (uint64_t)p.T * p.k;
-    act_src[1] = p.x;
+    act_src[1] = xg + (size_t)p.T * p.k * p.d;
     act_rows[1] = p.T;
   } else {
     act_src[0] = p.h;
@@ -611,17 +785,19 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
     for (int bx = 0; bx < kBoxes; ++bx) {
       const uint32_t rows = (uint32_t)std::min<uint64_t>(16u << bx, act_rows[s]);
       maps.box_rows[s][bx] = (int)rows;
-      if (!make_map(&maps.act[s][bx], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act_src[s], K,
+      if (!make_map(&maps.act[s][bx], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, act_src[s], K,
                     act_rows[s], kTcBK, rows, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     }
   }
   auto kern = tc_grouped_kernel<FMT, GATE_UP>;
+  const int smem = tc_smem<FMT, GATE_UP>(K, p.E).total;
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int sms = 0;
   std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     int dev = 0;
     if (attr_err == cudaSuccess) attr_err = cudaGetDevice(&dev);
     if (attr_err == cudaSuccess)
@@ -631,7 +807,7 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);
   cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -657,7 +833,7 @@ bool tc_supported(const Plan& p) {
 }
 
 cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st) {
-  const long long work = (long long)p.T * p.k * (p.d / 8);
+  const long long work = ((long long)p.T * p.k + p.T) * (p.d / 8);
   const int blocks = (int)std::max(1LL, std::min<long long>(1184, (work + 255) / 256));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
