@@ -18,7 +18,8 @@ PATH_CODE = {"auto": 0, "gemv": 1, "tc": 2}
 N_MARKS = 6
 
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error",
-          -4: "device timeout", -5: "workspace", -6: "device check failed"}
+          -4: "device timeout", -5: "workspace", -6: "device check failed",
+          -7: "too large for the built-in scratch"}
 
 
 class MoeError(RuntimeError):
@@ -44,7 +45,8 @@ class MoeLayer(ctypes.Structure):
 _LIB = None
 EXPORTS = ["moe_abi_version", "moe_status_str", "moe_validate", "moe_workspace_size",
            "moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
-           "moe_layer_forward_marked", "moe_device_status", "moe_launches_per_call"]
+           "moe_layer_forward_marked", "moe_device_status", "moe_launches_per_call",
+           "moe_layer_forward_static"]
 
 
 def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
@@ -75,6 +77,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
                                            ctypes.POINTER(P), I32]),
         "moe_device_status": (I32, [LP, P, SZ, ctypes.POINTER(I32), P]),
         "moe_launches_per_call": (I32, [LP]),
+        "moe_layer_forward_static": (I32, [LP, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -247,3 +250,15 @@ def device_status(L: MoeLayer, ws, stream=None) -> int:
                                             ctypes.byref(code), _stream(stream)),
            "moe_device_status")
     return code.value
+
+
+def layer_forward_static(L: MoeLayer, x, out=None, stream=None):
+    """The layer with the library's built-in scratch (no workspace argument): for callers
+    that cannot allocate device memory. Limits and sharing rules: include/moe_b200.h."""
+    import torch
+    if out is None:
+        out = torch.empty((L.T, L.d), dtype=torch.bfloat16, device=x.device)
+    _check(load_library().moe_layer_forward_static(ctypes.byref(L), x.data_ptr(),
+                                                   out.data_ptr(), _stream(stream)),
+           "moe_layer_forward_static")
+    return out

@@ -221,6 +221,7 @@ const char* moe_status_str(int32_t s) {
     case MOE_ERR_TIMEOUT: return "device-side wait timed out";
     case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case MOE_ERR_DEVICE: return "device-side check failed";
+    case MOE_ERR_TOO_LARGE: return "request exceeds the library's built-in scratch buffer";
     default: return "unknown status";
   }
 }

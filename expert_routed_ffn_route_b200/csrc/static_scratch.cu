@@ -1,0 +1,48 @@
+// moe_layer_forward_static: the layer for callers that cannot allocate device memory.
+// The intermediates live in a scratch buffer owned by the library (a file-scope device
+// array, present on every GPU that loads the library until the process exits), so the call
+// allocates and frees nothing. See include/moe_b200.h for the limits and the sharing rules.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace {
+
+static __device__ __align__(256) uint8_t g_static_scratch[MOE_STATIC_SCRATCH_BYTES];
+
+// Device address of the scratch on each device, looked up once per device with that
+// device current (the array's name in host code is only a stand-in for the symbol).
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+moe_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_layer_forward_static(const moe_layer* L, const void* x, void* out,
+                                               moe_stream_t stream) {
+  moe_status s = moe_validate(L);
+  if (s != MOE_OK) return s;
+  const size_t need = moe_workspace_size(L);
+  if (need == 0) return MOE_ERR_INVALID_ARG;
+  if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_TOO_LARGE;
+  void* ws = nullptr;
+  if ((s = scratch_address(&ws)) != MOE_OK) return s;
+  // the status word and the routing ticket at the start of the workspace begin at zero
+  if (cudaMemsetAsync(ws, 0, 256, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return moe_layer_forward(L, x, out, nullptr, nullptr, nullptr, nullptr, ws,
+                           MOE_STATIC_SCRATCH_BYTES, stream);
+}

@@ -66,7 +66,8 @@ typedef enum {
   MOE_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch or attribute)       */
   MOE_ERR_TIMEOUT = -4,     /* a bounded device-side wait gave up (device status)     */
   MOE_ERR_WORKSPACE = -5,   /* workspace NULL, misaligned or smaller than required    */
-  MOE_ERR_DEVICE = -6       /* a device-side check failed (see moe_device_status)     */
+  MOE_ERR_DEVICE = -6,      /* a device-side check failed (see moe_device_status)     */
+  MOE_ERR_TOO_LARGE = -7    /* the request needs more than the library's built-in scratch */
 } moe_status;
 
 typedef enum { MOE_W_BF16 = 16, MOE_W_INT8 = 8, MOE_W_INT4 = 4 } moe_wfmt;
@@ -168,6 +169,32 @@ MOE_API int32_t moe_launches_per_call(const moe_layer* L);
  * the code to *code (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE) and clears it. */
 MOE_API moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,
                              moe_stream_t stream);
+
+/* For callers that cannot allocate device memory. Some callers have no way to call
+ * cudaMalloc when the layer runs: code running inside a stream-ordered region whose
+ * allocator is owned by someone else, plug-ins that are handed a stream but no allocator,
+ * or processes with a fixed device-memory budget that was reserved up front. This entry
+ * point runs the same layer as moe_layer_forward (same kernels, same result) but keeps
+ * every intermediate in a scratch buffer that lives inside the library itself: a
+ * 16 MiB array in device memory, part of the library's image on every GPU that loads it
+ * and held until the process exits. It allocates nothing and frees nothing.
+ *
+ *   - Limit: the call's moe_workspace_size(L) must be at most MOE_STATIC_SCRATCH_BYTES
+ *     (16 MiB; it covers decode and verify calls of up to 32 tokens at d <= 4096,
+ *     f <= 2048, E <= 1024, k <= 16). Larger requests return MOE_ERR_TOO_LARGE and enqueue
+ *     nothing.
+ *   - The first call on a device looks up the buffer's device address (once per device);
+ *     make that first call before capturing a stream into a CUDA graph.
+ *   - Every call on a device shares the one buffer, and it keeps the previous call's
+ *     contents (the call clears the words that must start at zero). Calls that can run at
+ *     the same time on one device (different streams, or different host threads without
+ *     ordering) race on it and give wrong results; order them on one stream.
+ *   - x and out as for moe_layer_forward; the routing outputs are not returned.
+ * This entry point has no counterpart in the pages the layer follows; it is a deployment
+ * aid of this library. */
+#define MOE_STATIC_SCRATCH_BYTES (16u << 20)
+MOE_API moe_status moe_layer_forward_static(const moe_layer* L, const void* x, void* out,
+                                            moe_stream_t stream);
 
 #ifdef __cplusplus
 }
