@@ -67,6 +67,43 @@ def bank_bytes_per_expert(cfg):
     return w, s
 
 
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of per-rank values over the process group (the job is as fast as its
+    slowest rank); identity without a process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def kernel_source_digest():
+    """Digest of the sources of the dominant decode kernel (ties ncu counters to a build)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemv_tma.cu", "gemv_frag.cu", "pipeline.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "expert_routed_ffn_route_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if it was
+    captured from the current kernel sources (else None)."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"gemv_tma_gate_up_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.]+)", text)
+    d = re.search(r"source_digest:\s*([0-9a-f]+)", text)
+    if not m or not d or d.group(1) != kernel_source_digest():
+        return None
+    return float(m.group(1))
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 def cpu_oracle_rate(cfg, L, seconds):
@@ -323,10 +360,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1) / e_steps
     status = B.device_status(descs[0], ws)
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
 
     peak, peak_kind = measured_peaks()
     ms_per_step = ms / args.steps
@@ -350,7 +384,8 @@ def run_ours(args, rank, world, local_rank):
                    "cuda_graph": not args.no_graph},
         "roofline": {"bound": "hbm", "kernel": "grouped gate/up + SwiGLU",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": profiled_traffic(cfg.name),
                      "avg_launch_ms": gu_avg_ms,
                      "layer_frac": float(np.mean(layer_bytes)) / (ms_per_step * 1e-3) / 1e9 / peak},
         "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",

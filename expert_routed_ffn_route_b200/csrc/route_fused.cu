@@ -11,8 +11,6 @@
 // (Qwen3.8-Flash-Next-Dual-GPU README, "Independent decode lane"); gates = softmax over the
 // selected logits; plan = counts, exclusive scan, stable scatter (README, "Dedicated
 // prefill lane", step 1).
-#include <cstdlib>
-
 #include "pipeline.cuh"
 
 namespace moe {
@@ -280,10 +278,7 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
 bool route_fused_supported(const Plan& p) { return p.T <= kRFMaxT && p.E <= kMaxE; }
 
 cudaError_t launch_route_fused(const Plan& p, int32_t* ticket, cudaStream_t st) {
-  int blocks = (p.E + kRFWarps - 1) / kRFWarps;
-#ifdef MOE_TRACE
-  if (const char* b = getenv("MOE_RF_BLOCKS")) blocks = atoi(b);
-#endif
+  const int blocks = (p.E + kRFWarps - 1) / kRFWarps;
   route_fused_kernel<<<blocks, kRFThreads, 0, st>>>(p, ticket);
   return cudaGetLastError();
 }
