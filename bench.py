@@ -79,27 +79,34 @@ def max_over_ranks(values, device="cpu"):
     return [float(v) for v in t.tolist()]
 
 
-def kernel_source_digest():
-    """Digest of the sources of the dominant decode kernel (ties ncu counters to a build)."""
+KERNEL_SOURCES = {
+    "gemv_tma": ("gemv_tma.cu", "gemv_frag.cuh", "pipeline.cuh", "common.cuh"),
+    "tc_grouped": ("tc_grouped.cu", "pipeline.cuh", "common.cuh"),
+}
+
+
+def kernel_source_digest(kernel="gemv_tma"):
+    """Digest of the sources of one gate/up kernel (ties committed ncu counters to a build)."""
     import hashlib
     h = hashlib.sha256()
-    for f in ("gemv_tma.cu", "gemv_frag.cu", "pipeline.cuh", "common.cuh"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "expert_routed_ffn_route_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if it was
-    captured from the current kernel sources (else None)."""
+def profiled_traffic(workload, kernel="gemv_tma"):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary
+    ``profiles/<kernel>_gate_up_<workload>.md``, if it was captured from the current kernel
+    sources (else None)."""
     import re
-    path = os.path.join(ROOT, "profiles", f"gemv_tma_gate_up_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_gate_up_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.]+)", text)
     d = re.search(r"source_digest:\s*([0-9a-f]+)", text)
-    if not m or not d or d.group(1) != kernel_source_digest():
+    if not m or not d or d.group(1) != kernel_source_digest(kernel):
         return None
     return float(m.group(1))
 
@@ -385,7 +392,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": "grouped gate/up + SwiGLU",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": profiled_traffic(cfg.name),
+                     "traffic": profiled_traffic(cfg.name,
+                                                 "tc_grouped" if cfg.T > 32 else "gemv_tma"),
                      "avg_launch_ms": gu_avg_ms,
                      "layer_frac": float(np.mean(layer_bytes)) / (ms_per_step * 1e-3) / 1e9 / peak},
         "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
