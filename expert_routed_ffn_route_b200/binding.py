@@ -14,7 +14,7 @@ import numpy as np
 from . import _build
 
 FMT_CODE = {"bf16": 16, "int8": 8, "int4": 4}
-PATH_CODE = {"auto": 0, "gemv": 1, "tc": 2}
+PATH_CODE = {"auto": 0, "gemv": 1, "tc": 2, "fused": 3}
 N_MARKS = 6
 
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error",

@@ -155,6 +155,8 @@ struct Plan {
   float* y_shared;     // [T*d]
   int32_t* status;
   int32_t* ticket;     // zero between calls; the fused routing kernel's completion counter
+  uint32_t* gbar;      // grid-barrier word of the single-kernel 1-token path (any value)
+  int32_t* tile_cnt;   // [d / 16] per-output-tile arrival counters, zero between calls
   uint16_t* xg;        // tensor-core path: fp16 x rows in grouped order, then the shared
                        // expert's rows [(T*k + T)][d]
   int32_t* tc_sched;   // tensor-core path: per-slot schedule (TcSched view)
@@ -171,6 +173,10 @@ struct TcSched {
   int32_t* slot_expert;  // [E + 2]
   int32_t* mt_prefix;    // [E + 2]; mt_prefix[n_slots] = total m-tiles
 };
+
+// The synchronisation block at the start of the workspace: status word (offset 0), routing
+// ticket (16), grid-barrier word (32), then one arrival counter per 16-row output tile (256).
+inline size_t sync_bytes(int d) { return 256 + (size_t)4 * (d / 16); }
 
 // Permutation chunking (assignments per scatter CTA).
 constexpr int kPermChunk = 256;
@@ -196,6 +202,10 @@ cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaSt
 cudaError_t launch_tc_gate_up(const Plan& p, const TcSched& S, const uint16_t* xg,
                               cudaStream_t st);
 cudaError_t launch_tc_down(const Plan& p, const TcSched& S, cudaStream_t st);
+// the whole layer of a 1-token call in one persistent kernel (decode_fused.cu)
+bool decode_fused_supported(const Plan& p);
+cudaError_t launch_decode_fused(const Plan& p, void* out, uint32_t* gbar, int32_t* tile_cnt,
+                                cudaStream_t st);
 // router + top-k + plan in one launch (T <= 32)
 bool route_fused_supported(const Plan& p);
 cudaError_t launch_route_fused(const Plan& p, int32_t* ticket, cudaStream_t st);

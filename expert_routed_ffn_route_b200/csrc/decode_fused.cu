@@ -1,0 +1,709 @@
+// The whole layer for a 1-token call in ONE persistent kernel (one CTA per SM, launched
+// cooperatively so that every CTA is resident and grid-wide barriers are safe).
+//
+// A decode token reads ~47 MB of weights in a few microseconds; separate launches for
+// routing, gate/up, down and combine cost more than the weight streaming itself. Here the
+// phases run back to back inside one grid, and every weight byte that does not depend on
+// the routing decision (router rows, the shared expert) is already in flight before that
+// decision is known:
+//
+//   prologue   each CTA issues bulk copies (TMA engine, no multicast) of its slice of the
+//              router rows and of its shared-expert gate/up tile, and an L2 prefetch of its
+//              shared-expert down rows.
+//   route      logits of the CTA's router rows -> workspace; grid barrier B1 (the CTA's
+//              shared-expert tile is multiplied while the barrier settles); then EVERY CTA
+//              reads the E logits and runs the same stable top-k and softmax over the picks
+//              (no second barrier: all CTAs reach the same decision from the same data).
+//   gate/up    the CTA's routed gate/up tiles (16 rows of one expert's gate and up, with
+//              their group scales) are all requested at once, and the L2 prefetch of its
+//              routed down rows follows them; h = silu(Wg x) * (Wu x) per row, rounded to
+//              bf16, is written to the workspace. Grid barrier B2.
+//   down       the CTA's down units (16 output rows of one expert) were copied into the
+//              freed tile buffers before B2; y = Wd h per unit in fp32 -> workspace.
+//   combine    per 16-row output tile, the CTA that completes it (an arrival counter per
+//              tile, no waiting) sums out = sum_j gate_j * y_j + y_shared in the fixed
+//              order j = 0..k-1, then the shared term, and rounds once to bf16.
+//
+// Products run on the tensor cores (mma.sync m16n8k16, weights as the 16-row A operand,
+// the token as column 0 of B), with the int4 codes entering exactly (gemv_frag.cuh) and the
+// group scale applied to the fp32 partial of each 128-wide K group. Every K-group partial
+// is reduced across warps in a fixed order, so the result is bitwise reproducible.
+//
+// What is computed is the layer of include/moe_b200.h: stable top-k with ties to the lower
+// index (Qwen3.8-Flash-Next-Dual-GPU README, "Independent decode lane"), SwiGLU experts on
+// symmetric group-128 int4 weights ("Model artifact and memory placement"), a fixed-order
+// reduction of each token's routes without atomics on the data ("Dedicated prefill lane",
+// step 5), unselected experts never read (TandemLLM docs, "17 Qwen3.8-Flash-Next", §17.4).
+#include <mutex>
+
+#include "gemv_frag.cuh"
+#include "pipeline.cuh"
+
+namespace moe {
+
+constexpr int kDfWarps = 20;                 // compute warps
+constexpr int kDfCompute = 32 * kDfWarps;
+constexpr int kDfThreads = kDfCompute + 32;  // + the producer warp
+constexpr int kDfRows = 16;                  // weight rows of a tile / unit (MMA M)
+constexpr int kDfMaxTiles = 8;
+constexpr int kDfMaxUnits = 24;
+constexpr int kDfMaxRouter = 8;
+
+#ifdef MOE_TRACE
+__device__ long long g_dftrace[160][16];
+#define DFT(slot) \
+  do { if (threadIdx.x == 0 && blockIdx.x < 160) { unsigned long long _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_dftrace[blockIdx.x][(slot)] = (long long)_t; } } while (0)
+extern "C" __attribute__((visibility("default"))) int moe_dftrace_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_dftrace, sizeof(g_dftrace));
+}
+#define DFTP(slot) \
+  do { if (blockIdx.x < 160) { unsigned long long _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_dftrace[blockIdx.x][(slot)] = (long long)_t; } } while (0)
+#else
+#define DFT(slot) do {} while (0)
+#define DFTP(slot) do {} while (0)
+#endif
+
+// Smem scratch beyond the buffers: picks, gates and the CTA's tile/unit tables.
+struct DfMisc {
+  int sel[kMaxK];
+  float gate[kMaxK];
+  int tile_slot[kDfMaxTiles], tile_rt[kDfMaxTiles];
+  int unit_slot[kDfMaxUnits], unit_rt[kDfMaxUnits];
+  int n_tiles, n_units, first_routed, ok, n_combine, armed_tiles, armed_units, armed_h;
+  int combine_rt[kDfMaxUnits];
+};
+
+// Shared-memory plan of one launch (identical on the host and in every CTA).
+struct DfLayout {
+  int grid, n_slots, G, Gf;
+  int tiles_total, tiles_max, units_total, units_max, router_max;
+  uint32_t tile_bytes, unit_bytes;
+  uint32_t off_router, off_h, off_x, off_xsum, off_red, off_bar, off_misc, total;
+};
+
+__host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int k,
+                                              int has_shared) {
+  DfLayout L;
+  L.grid = grid;
+  L.n_slots = k + has_shared;
+  L.G = d / kGroup;
+  L.Gf = f / kGroup;
+  L.tiles_total = L.n_slots * (f / kDfRows);
+  L.tiles_max = (L.tiles_total + grid - 1) / grid;
+  L.units_total = L.n_slots * (d / kDfRows);
+  L.units_max = (L.units_total + grid - 1) / grid;
+  L.router_max = (E + grid - 1) / grid;
+  // gate and up rows (int4) then their bf16 scales
+  L.tile_bytes = 2u * kDfRows * (d / 2) + 2u * kDfRows * L.G * 2;
+  L.unit_bytes = (uint32_t)kDfRows * (f / 2) + (uint32_t)kDfRows * L.Gf * 2;
+  // one region holds the gate/up tiles, later the down units; the router rows alias its end
+  // when they leave buffer 0 (the shared tile, copied meanwhile) free, else follow it
+  const uint32_t router_bytes = (uint32_t)L.router_max * d * 2;
+  // the h rows of the call (staged after B2) follow the down units
+  L.off_h = L.units_max * L.unit_bytes;
+  uint32_t region = max(L.tiles_max * L.tile_bytes, L.off_h + (uint32_t)L.n_slots * f * 2);
+  if (router_bytes + (has_shared ? L.tile_bytes : 0u) <= region) {
+    L.off_router = region - router_bytes;
+  } else {
+    L.off_router = region;
+    region += router_bytes;
+  }
+  uint32_t o = region;
+  L.off_x = o;
+  o += 2u * d;
+  L.off_xsum = o;
+  o += 4u * L.G;
+  o = (o + 15) & ~15u;
+  L.off_red = o;
+  uint32_t red_gu = (uint32_t)L.tiles_max * 2 * L.G * kDfRows * 4;
+  uint32_t red_dn = (uint32_t)L.units_max * L.Gf * kDfRows * 4;
+  uint32_t red_rt = (uint32_t)kDfMaxRouter * L.G * 4;
+  o += max(red_gu, max(red_dn, red_rt));
+  o = (o + 15) & ~15u;
+  L.off_bar = o;
+  o += 8u * (2 + kDfMaxTiles + kDfMaxUnits);
+  L.off_misc = o;
+  o += (uint32_t)((sizeof(DfMisc) + 15) & ~size_t(15));
+  L.total = o;
+  return L;
+}
+
+// ------------------------------------------------------------------ grid barrier
+
+// Grid-wide barrier on one 32-bit word whose low 31 bits are zero between barriers (the
+// workspace starts zeroed). Every CTA adds to the word once per barrier; CTA 0 adds
+// 2^31 - (grid - 1) and the others 1, so the top bit flips exactly when the last CTA
+// arrives and the low bits are zero again afterwards. A CTA is through once it sees the
+// top bit differ from the value it found on arrival.
+__device__ __forceinline__ uint32_t gbar_arrive(uint32_t* bar) {
+  const uint32_t add = (blockIdx.x == 0) ? (0x80000000u - (gridDim.x - 1)) : 1u;
+  __threadfence();
+  return atomicAdd(bar, add);
+}
+
+__device__ __forceinline__ bool gbar_wait(const uint32_t* bar, uint32_t arrived) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t now;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(bar) : "memory");
+    if ((now ^ arrived) & 0x80000000u) break;
+    if (clock64() - t0 > kWaitCycles) return false;
+    __nanosleep(32);
+  }
+  __threadfence();
+  return true;
+}
+
+// A wait that every lane of the warp leaves with the same verdict.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar) {
+  const bool ok = mbar_wait(bar, 0);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// ------------------------------------------------------------------ tile products
+
+// One 128-wide K group of a 16-row int4 tile against one activation row held as the
+// B operand's column 0 (xb: the lane's 32 activation values of the group, permuted into
+// fragment order; zero on lanes that do not carry column 0). Returns, on lanes with q == 0,
+// the biased dot products of rows grp and grp + 8 (codes enter as q + 136).
+__device__ __forceinline__ void t1_group(const uint8_t* tile, uint32_t row_bytes, int g, int grp,
+                                         int q, const uint32_t (&xb)[16], float& ra,
+                                         float& rb) {
+  uint4 wa[1], wb[1];
+  wa[0] = *reinterpret_cast<const uint4*>(tile + grp * row_bytes + g * 64 + q * 16);
+  wb[0] = *reinterpret_cast<const uint4*>(tile + (grp + 8) * row_bytes + g * 64 + q * 16);
+  uint32_t fa[8][2], fb[8][2];
+  to_frags<4>(wa, fa);
+  to_frags<4>(wb, fb);
+  float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int m = 0; m < 8; m += 2) {
+    mma_bf16_16x8x16(c0, fa[m][0], fb[m][0], fa[m][1], fb[m][1], xb[2 * m], xb[2 * m + 1]);
+    mma_bf16_16x8x16(c1, fa[m + 1][0], fb[m + 1][0], fa[m + 1][1], fb[m + 1][1],
+                     xb[2 * m + 2], xb[2 * m + 3]);
+  }
+  ra = c0[0] + c1[0];
+  rb = c0[2] + c1[2];
+}
+
+// The lane's 32 activation values [32 q, 32 q + 32) of group g of a bf16 row, in fragment
+// order, and their sum (fixed order: within the lane, then across the 4 lanes of the row).
+template <bool GLOBAL>
+__device__ __forceinline__ float t1_load_act(const uint16_t* row, int g, int q, bool carry,
+                                             uint32_t (&xb)[16]) {
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (carry) {
+      const uint4* src = reinterpret_cast<const uint4*>(row + g * kGroup + 32 * q + 8 * i);
+      v = GLOBAL ? __ldcg(src) : *src;
+    }
+    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      s += __uint_as_float(vv[j] << 16);
+      s += __uint_as_float(vv[j] & 0xffff0000u);
+    }
+    permute_chunk<4>(v);
+    xb[4 * i + 0] = v.x;
+    xb[4 * i + 1] = v.y;
+    xb[4 * i + 2] = v.z;
+    xb[4 * i + 3] = v.w;
+  }
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  return s;
+}
+
+// ------------------------------------------------------------------ the kernel
+
+// Warps 0..kDfWarps-1 compute; warp kDfWarps (the producer) issues every bulk copy and L2
+// prefetch (one lane a copy) and spins on the grid barriers, so no compute warp stalls on
+// copy issue or on another CTA.
+__global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uint16_t* out,
+                                                                     uint32_t* gbar,
+                                                                     int32_t* tile_cnt) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int d = p.d, f = p.f, E = p.E, k = p.k;
+  const DfLayout L = df_layout(gridDim.x, d, f, E, k, p.has_shared);
+  const int G = L.G, Gf = L.Gf, S = L.n_slots;
+  const uint32_t rowb_up = d / 2, rowb_dn = f / 2;
+  uint16_t* s_x = reinterpret_cast<uint16_t*>(smem + L.off_x);
+  float* s_xsum = reinterpret_cast<float*>(smem + L.off_xsum);
+  float* red = reinterpret_cast<float*>(smem + L.off_red);
+  const uint16_t* s_h = reinterpret_cast<const uint16_t*>(smem + L.off_h);
+  uint64_t* bar_router = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+  uint64_t* bar_h = bar_router + 1;
+  uint64_t* bar_tile = bar_router + 2;
+  uint64_t* bar_unit = bar_tile + kDfMaxTiles;
+  DfMisc* mi = reinterpret_cast<DfMisc*>(smem + L.off_misc);
+  const uint16_t* s_router = reinterpret_cast<const uint16_t*>(smem + L.off_router);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = (warp == kDfWarps);
+  const int grp = lane >> 2, q = lane & 3;
+  const int c = blockIdx.x, grid = gridDim.x;
+  const int r0 = (int)((long long)E * c / grid), r1 = (int)((long long)E * (c + 1) / grid);
+  const int nr = r1 - r0;
+  DFT(0);
+
+  // ---------------------------------------------------------------- prologue
+  if (producer) {
+    if (lane == 0) {
+      mbar_init(bar_router, 1);
+      mbar_init(bar_h, 1);
+      for (int i = 0; i < kDfMaxTiles; ++i) mbar_init(&bar_tile[i], 1);
+      for (int i = 0; i < kDfMaxUnits; ++i) mbar_init(&bar_unit[i], 1);
+      fence_barrier_init();
+      // first the copies that do not depend on anything: the router rows of this CTA and
+      // its shared-expert tile (at most one: tiles are numbered with the slot fastest)
+      const uint32_t rb = (uint32_t)nr * d * 2;
+      mbar_arrive_expect_tx(bar_router, rb);
+      if (rb) bulk_g2s(smem + L.off_router, p.router_w + (size_t)r0 * d, rb, bar_router);
+      const int t0 = (int)((long long)L.tiles_total * c / grid);
+      const int t1 = (int)((long long)L.tiles_total * (c + 1) / grid);
+      const int sh_i = p.has_shared ? (t0 + S - 1) / S * S : t1;  // first multiple of S >= t0
+      const bool has_sh_tile = sh_i < t1;
+      if (has_sh_tile) {
+        const size_t row = (size_t)(sh_i / S) * kDfRows;
+        const uint32_t wbytes = kDfRows * rowb_up, sbytes = kDfRows * G * 2;
+        mbar_arrive_expect_tx(&bar_tile[0], L.tile_bytes);
+        bulk_g2s(smem, static_cast<const uint8_t*>(p.shared.w[0]) + row * rowb_up, wbytes, &bar_tile[0]);
+        bulk_g2s(smem + wbytes, static_cast<const uint8_t*>(p.shared.w[1]) + row * rowb_up, wbytes,
+                 &bar_tile[0]);
+        bulk_g2s(smem + 2 * wbytes, p.shared.s[0] + row * G, sbytes, &bar_tile[0]);
+        bulk_g2s(smem + 2 * wbytes + sbytes, p.shared.s[1] + row * G, sbytes, &bar_tile[0]);
+      }
+      // tile table: the shared tile (if any) first, in buffer 0; routed tiles after it
+      int n = 0;
+      if (has_sh_tile) { mi->tile_slot[0] = 0; mi->tile_rt[0] = sh_i / S; n = 1; }
+      mi->first_routed = n;
+      for (int i = t0; i < t1; ++i)
+        if (i != sh_i) { mi->tile_slot[n] = i % S; mi->tile_rt[n] = i / S; ++n; }
+      mi->n_tiles = n;
+      const int u0 = (int)((long long)L.units_total * c / grid);
+      const int u1 = (int)((long long)L.units_total * (c + 1) / grid);
+      for (int i = u0; i < u1; ++i) { mi->unit_slot[i - u0] = i % S; mi->unit_rt[i - u0] = i / S; }
+      mi->n_units = u1 - u0;
+      mi->ok = 1;
+      mi->armed_tiles = has_sh_tile ? 1 : 0;
+      mi->armed_units = 0;
+      mi->armed_h = 0;
+      if (p.has_shared)
+        for (int i = 0; i < mi->n_units; ++i)
+          if (mi->unit_slot[i] == 0) {
+            const size_t row = (size_t)mi->unit_rt[i] * kDfRows;
+            prefetch_l2(static_cast<const uint8_t*>(p.shared.w[2]) + row * rowb_dn, kDfRows * rowb_dn);
+            prefetch_l2(p.shared.s[2] + row * Gf, kDfRows * Gf * 2);
+          }
+    }
+    __syncwarp();
+  } else {
+    // the activation row (bf16)
+    for (int i = tid; i < d / 8; i += kDfCompute)
+      reinterpret_cast<uint4*>(s_x)[i] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+  }
+  __syncthreads();  // S1: tables, barriers and x
+
+  // ---------------------------------------------------------------- router logits
+  if (!producer) {
+    for (int g = warp; g < G; g += kDfWarps) {  // per-group sums of x
+      const uint2 v = *reinterpret_cast<const uint2*>(s_x + g * kGroup + 4 * lane);
+      float s = __uint_as_float(v.x << 16);
+      s += __uint_as_float(v.x & 0xffff0000u);
+      s += __uint_as_float(v.y << 16);
+      s += __uint_as_float(v.y & 0xffff0000u);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) s_xsum[g] = s;
+    }
+    DFT(1);
+    if (!mbar_wait(bar_router, 0)) {
+      set_status(p.status, DEV_TIMEOUT);
+      mi->ok = 0;
+    }
+    DFT(2);
+    for (int g = warp; g < G; g += kDfWarps) {
+      const uint2 xv = *reinterpret_cast<const uint2*>(s_x + g * kGroup + 4 * lane);
+      const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+      const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
+      for (int r = 0; r < nr; ++r) {
+        const uint2 wv = *reinterpret_cast<const uint2*>(s_router + (size_t)r * d + g * kGroup + 4 * lane);
+        float s = x0 * __uint_as_float(wv.x << 16);
+        s = fmaf(x1, __uint_as_float(wv.x & 0xffff0000u), s);
+        s = fmaf(x2, __uint_as_float(wv.y << 16), s);
+        s = fmaf(x3, __uint_as_float(wv.y & 0xffff0000u), s);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) red[r * G + g] = s;
+      }
+    }
+    named_bar_sync(1, kDfCompute);
+    if (tid < nr) {
+      float s = 0.f;
+      for (int g = 0; g < G; ++g) s += red[tid * G + g];
+      const int e = r0 + tid;
+      p.logits[e] = s + (p.router_bias ? p.router_bias[e] : 0.f);
+    }
+  }
+  __syncthreads();  // S2: this CTA's logits are written
+  DFT(3);
+
+  // Items (tile position b, matrix m, group g), warp w takes every kDfWarps-th item of a
+  // tile range; partials land in red[b][m][g][16] (rows of the tile), scaled and corrected.
+  auto gate_up_items = [&](int b_begin, int b_end) {
+    int cur_g = -1;
+    uint32_t xb[16];
+    float corr = 0.f;
+    for (int b = b_begin; b < b_end; ++b) {
+      if (warp >= 2 * G) break;
+      if (!warp_wait(&bar_tile[b])) {
+        if (lane == 0) set_status(p.status, DEV_TIMEOUT);
+        return;
+      }
+#ifdef MOE_TRACE
+      if (warp == 0 && b == mi->first_routed) DFT(8);
+#endif
+      const uint8_t* tile = smem + (size_t)b * L.tile_bytes;
+      const uint16_t* scales = reinterpret_cast<const uint16_t*>(tile + 2 * kDfRows * rowb_up);
+      float* red_b = red + (size_t)b * 2 * G * kDfRows;
+      for (int r = warp; r < 2 * G; r += kDfWarps) {
+        const int m = (r >= G) ? 1 : 0, g = r - m * G;
+        if (g != cur_g) {
+          t1_load_act<false>(s_x, g, q, grp == 0, xb);
+          corr = 136.f * s_xsum[g];
+          cur_g = g;
+        }
+        float ra, rb;
+        t1_group(tile + m * kDfRows * rowb_up, rowb_up, g, grp, q, xb, ra, rb);
+        if (q == 0) {
+          const uint16_t* sc = scales + m * kDfRows * G + g;
+          float* dst = red_b + (size_t)r * kDfRows;
+          dst[grp] = bf16_to_f32(sc[grp * G]) * (ra - corr);
+          dst[grp + 8] = bf16_to_f32(sc[(grp + 8) * G]) * (rb - corr);
+        }
+      }
+    }
+  };
+
+  // ---------------------------------------------------------------- B1 (+ the shared tile)
+  __shared__ uint32_t s_arrived;
+  if (producer) {
+    if (lane == 0) {
+      s_arrived = gbar_arrive(gbar);
+      if (mi->ok && !gbar_wait(gbar, s_arrived)) {
+        set_status(p.status, DEV_TIMEOUT);
+        mi->ok = 0;
+      }
+      DFTP(4);
+    }
+    __syncwarp();  // the warp reaches the CTA barrier converged
+  } else if (mi->ok) {
+    gate_up_items(0, mi->first_routed);  // the shared tile, while B1 settles
+  }
+  __syncthreads();  // S3
+  DFT(5);
+
+  // ---------------------------------------------------------------- top-k (every CTA)
+  if (mi->ok && warp == 0) {
+    int e;
+    uint32_t key;
+    DFT(7);
+    warp_topk(p.logits, E, k, lane, &e, &key);
+    DFT(12);
+    const uint32_t top = __shfl_sync(0xffffffffu, key, 0);
+    const float gte = warp_topk_gate(key, top, k, lane);
+    if (lane < k) {
+      mi->sel[lane] = e;
+      mi->gate[lane] = gte;
+    }
+  }
+  __syncthreads();  // S4: the routing decision
+  DFT(6);
+  const bool ok1 = mi->ok;
+
+  // ---------------------------------------------------------------- gate/up tiles
+  if (producer) {
+    if (ok1) {
+      // routed tiles, one lane a tile (the router rows they overwrite are consumed)
+      fence_proxy_async();
+      const int b = mi->first_routed + lane;
+      if (b < mi->n_tiles) {
+        const uint32_t wbytes = kDfRows * rowb_up, sbytes = kDfRows * G * 2;
+        const int j = mi->tile_slot[b] - p.has_shared;
+        const size_t row = (size_t)mi->sel[j] * f + (size_t)mi->tile_rt[b] * kDfRows;
+        uint8_t* dst = smem + (size_t)b * L.tile_bytes;
+        mbar_arrive_expect_tx(&bar_tile[b], L.tile_bytes);
+        bulk_g2s(dst, static_cast<const uint8_t*>(p.routed.w[0]) + row * rowb_up, wbytes, &bar_tile[b]);
+        bulk_g2s(dst + wbytes, static_cast<const uint8_t*>(p.routed.w[1]) + row * rowb_up, wbytes,
+                 &bar_tile[b]);
+        bulk_g2s(dst + 2 * wbytes, p.routed.s[0] + row * G, sbytes, &bar_tile[b]);
+        bulk_g2s(dst + 2 * wbytes + sbytes, p.routed.s[1] + row * G, sbytes, &bar_tile[b]);
+      }
+      if (lane == 0) mi->armed_tiles = mi->n_tiles;
+      __syncwarp();
+      // the routed down rows this CTA will need, into L2 behind the gate/up requests
+      for (int i = lane; i < mi->n_units; i += 32) {
+        const int slot = mi->unit_slot[i];
+        if (p.has_shared && slot == 0) continue;
+        const size_t row = (size_t)mi->sel[slot - p.has_shared] * d + (size_t)mi->unit_rt[i] * kDfRows;
+        prefetch_l2(static_cast<const uint8_t*>(p.routed.w[2]) + row * rowb_dn, kDfRows * rowb_dn);
+        prefetch_l2(p.routed.s[2] + row * Gf, kDfRows * Gf * 2);
+      }
+    }
+    __syncwarp();
+  } else if (ok1) {
+    if (c == 0) {  // the plan outputs of the call
+      if (tid < k) {
+        const int e = mi->sel[tid];
+        int rank = 0;
+        for (int j = 0; j < k; ++j) rank += (mi->sel[j] < e);
+        p.topk_idx[tid] = e;
+        p.topk_w[tid] = mi->gate[tid];
+        p.perm[rank] = tid;
+        p.inv[tid] = rank;
+      }
+      for (int e = tid; e <= E; e += kDfCompute) {
+        int cnt = 0;
+        for (int j = 0; j < k; ++j) cnt += (mi->sel[j] < e);
+        p.offsets[e] = cnt;
+      }
+    }
+    gate_up_items(mi->first_routed, mi->n_tiles);
+    DFT(9);
+  }
+  __syncthreads();  // S5: every gate/up product of this CTA is in red
+  DFT(10);
+
+  // h rows of this CTA's tiles: fixed-order sums over the K groups, SwiGLU, one rounding
+  if (ok1 && !producer) {
+    for (int i = tid; i < mi->n_tiles * kDfRows; i += kDfCompute) {
+      const int b = i / kDfRows, r = i % kDfRows;
+      const float* rg = red + (size_t)(b * 2) * G * kDfRows + r;
+      const float* ru = rg + (size_t)G * kDfRows;
+      float gs = 0.f, us = 0.f;
+      for (int g = 0; g < G; ++g) {
+        gs += rg[g * kDfRows];
+        us += ru[g * kDfRows];
+      }
+      const float hv = gs / (1.f + expf(-gs)) * us;
+      p.h[(size_t)mi->tile_slot[b] * f + (size_t)mi->tile_rt[b] * kDfRows + r] = f32_to_bf16_rn(hv);
+    }
+  }
+  __syncthreads();  // S6: h of this CTA written; the tile buffers are free
+  DFT(11);
+
+  // ---------------------------------------------------------------- B2
+  if (producer) {
+    if (ok1) {
+      // down units into the freed tile buffers (from L2 when the prefetch has landed)
+      fence_proxy_async();
+      for (int i = lane; i < mi->n_units; i += 32) {
+        const int slot = mi->unit_slot[i];
+        const bool sh = p.has_shared && slot == 0;
+        const Bank& bk = sh ? p.shared : p.routed;
+        const size_t e = sh ? 0 : (size_t)mi->sel[slot - p.has_shared];
+        const size_t row = e * d + (size_t)mi->unit_rt[i] * kDfRows;
+        const uint32_t wbytes = kDfRows * rowb_dn, sbytes = kDfRows * Gf * 2;
+        uint8_t* dst = smem + (size_t)i * L.unit_bytes;
+        mbar_arrive_expect_tx(&bar_unit[i], L.unit_bytes);
+        bulk_g2s(dst, static_cast<const uint8_t*>(bk.w[2]) + row * rowb_dn, wbytes, &bar_unit[i]);
+        bulk_g2s(dst + wbytes, bk.s[2] + row * Gf, sbytes, &bar_unit[i]);
+      }
+      if (lane == 0) mi->armed_units = mi->n_units;
+    }
+    // every CTA arrives at every barrier, failed or not, so the word stays consistent
+    if (lane == 0) {
+      s_arrived = gbar_arrive(gbar);
+      if (ok1 && !gbar_wait(gbar, s_arrived)) {
+        set_status(p.status, DEV_TIMEOUT);
+        mi->ok = 0;
+      }
+      if (mi->ok) {  // every h row of the call, into shared memory in one request
+        mbar_arrive_expect_tx(bar_h, (uint32_t)S * f * 2);
+        mi->armed_h = 1;
+      }
+    }
+    __syncwarp();
+    // the h rows were written through the generic proxy by other CTAs before B2
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    if (mi->ok)
+      for (int s = lane; s < S; s += 32)
+        bulk_g2s(smem + L.off_h + (size_t)s * f * 2, p.h + (size_t)s * f, f * 2, bar_h);
+    __syncwarp();
+  }
+  __syncthreads();  // S7: the B2 verdict
+  const bool ok2 = mi->ok;
+
+  // ---------------------------------------------------------------- down units
+  if (ok2 && !producer) {
+    if (!warp_wait(bar_h)) {
+      if (lane == 0) set_status(p.status, DEV_TIMEOUT);
+    } else {
+      uint32_t xb[16];
+      for (int u = 0; u < mi->n_units; ++u) {
+        const int slot = mi->unit_slot[u];
+        const uint8_t* unit = smem + (size_t)u * L.unit_bytes;
+        const uint16_t* scales = reinterpret_cast<const uint16_t*>(unit + kDfRows * rowb_dn);
+        // items (u, g) in one flat order over the CTA's units: warp w takes u * Gf + g = w mod W
+        const int first = ((warp - u * Gf) % kDfWarps + kDfWarps) % kDfWarps;
+        if (first >= Gf) continue;
+        if (!warp_wait(&bar_unit[u])) {
+          if (lane == 0) set_status(p.status, DEV_TIMEOUT);
+          break;
+        }
+        for (int g = first; g < Gf; g += kDfWarps) {
+          float hs = t1_load_act<false>(s_h + (size_t)slot * f, g, q, grp == 0, xb);
+          hs = __shfl_sync(0xffffffffu, hs, 0);
+          float ra, rb;
+          t1_group(unit, rowb_dn, g, grp, q, xb, ra, rb);
+          if (q == 0) {
+            const uint16_t* sc = scales + g;
+            const float corr = 136.f * hs;
+            float* dst = red + ((size_t)u * Gf + g) * kDfRows;
+            dst[grp] = bf16_to_f32(sc[grp * Gf]) * (ra - corr);
+            dst[grp + 8] = bf16_to_f32(sc[(grp + 8) * Gf]) * (rb - corr);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();  // S8
+  DFT(13);
+  if (ok2 && !producer) {
+    for (int i = tid; i < mi->n_units * kDfRows; i += kDfCompute) {
+      const int u = i / kDfRows, r = i % kDfRows;
+      const float* src = red + (size_t)u * Gf * kDfRows + r;
+      float y = 0.f;
+      for (int g = 0; g < Gf; ++g) y += src[g * kDfRows];
+      const int slot = mi->unit_slot[u];
+      const size_t n = (size_t)mi->unit_rt[u] * kDfRows + r;
+      if (p.has_shared && slot == 0) p.y_shared[n] = y;
+      else p.y_assign[(size_t)(slot - p.has_shared) * d + n] = y;
+    }
+  }
+  __syncthreads();  // S9: this CTA's y values written
+  if (producer) {
+    // Arrivals per output tile (one lane a tile; the CTA's units are consecutive, so each
+    // tile's units form one run). The CTA that completes a tile combines it.
+    const int nu = mi->n_units;
+    const int first_rt = nu ? mi->unit_rt[0] : 0;
+    const int rt = first_rt + lane;
+    int n = 0;
+    for (int i = 0; i < nu; ++i) n += (mi->unit_rt[i] == rt);
+    bool mine = false;
+    if (n > 0) {
+      __threadfence();
+      const int old = atomicAdd(&tile_cnt[rt], n);
+      if (old + n == S) {
+        tile_cnt[rt] = 0;  // every unit of the tile has arrived: ready for the next call
+        mine = ok2;
+        __threadfence();
+      }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, mine);
+    if (mine) mi->combine_rt[__popc(m & ((1u << lane) - 1u))] = rt;
+    if (lane == 0) mi->n_combine = __popc(m);
+  }
+  __syncthreads();  // S10
+  DFT(14);
+  if (ok2 && !producer) {
+    for (int i = tid; i < mi->n_combine * kDfRows; i += kDfCompute) {
+      const size_t n = (size_t)mi->combine_rt[i / kDfRows] * kDfRows + i % kDfRows;
+      float acc = 0.f;
+      for (int j = 0; j < k; ++j) acc = fmaf(mi->gate[j], __ldcg(p.y_assign + (size_t)j * d + n), acc);
+      if (p.has_shared) acc += __ldcg(p.y_shared + n);
+      out[n] = f32_to_bf16_rn(acc);
+    }
+  }
+  DFT(15);
+
+  // ---------------------------------------------------------------- drain
+  // No copy may land after the CTA ends: wait (boundedly) for every one that was issued.
+  // On the normal path every phase has completed already and each test is immediate.
+  if (producer && lane == 0) {
+    mbar_wait(bar_router, 0);
+    for (int b = 0; b < mi->armed_tiles; ++b) mbar_wait(&bar_tile[b], 0);
+    for (int u = 0; u < mi->armed_units; ++u) mbar_wait(&bar_unit[u], 0);
+    if (mi->armed_h) mbar_wait(bar_h, 0);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+struct DfCache {
+  std::mutex mu;
+  int dev = -1, sms = 0;
+  size_t smem_set = 0;
+};
+DfCache g_df;
+
+cudaError_t df_sms(int* sms) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(g_df.mu);
+  if (g_df.dev != dev) {
+    if ((err = cudaDeviceGetAttribute(&g_df.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return err;
+    g_df.dev = dev;
+    g_df.smem_set = 0;
+  }
+  *sms = g_df.sms;
+  return cudaSuccess;
+}
+}  // namespace
+
+bool decode_fused_supported(const Plan& p) {
+  if (p.T != 1 || p.routed.fmt != 4 || (p.has_shared && p.shared.fmt != 4)) return false;
+  if (p.k > 32 || p.E > kMaxE || p.d % kDfRows || p.f % kDfRows) return false;
+  int sms = 0;
+  if (df_sms(&sms) != cudaSuccess || sms < 1) return false;
+  const DfLayout L = df_layout(sms, p.d, p.f, p.E, p.k, p.has_shared);
+  if (L.tiles_max > kDfMaxTiles || L.units_max > kDfMaxUnits || L.router_max > kDfMaxRouter)
+    return false;
+  if (L.total > 227u * 1024u) return false;
+  // bulk copies: 16-byte aligned sources (scales too)
+  for (int i = 0; i < 3; ++i) {
+    if (reinterpret_cast<uintptr_t>(p.routed.s[i]) % 16) return false;
+    if (p.has_shared && reinterpret_cast<uintptr_t>(p.shared.s[i]) % 16) return false;
+  }
+  return true;
+}
+
+cudaError_t launch_decode_fused(const Plan& p, void* out, uint32_t* gbar, int32_t* tile_cnt,
+                                cudaStream_t st) {
+  int sms = 0;
+  cudaError_t err = df_sms(&sms);
+  if (err != cudaSuccess) return err;
+  const DfLayout L = df_layout(sms, p.d, p.f, p.E, p.k, p.has_shared);
+  {
+    std::lock_guard<std::mutex> lock(g_df.mu);
+    if (L.total > g_df.smem_set) {
+      err = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)L.total);
+      if (err != cudaSuccess) return err;
+      g_df.smem_set = L.total;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(kDfThreads);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_fused_kernel, p, static_cast<uint16_t*>(out), gbar,
+                            tile_cnt);
+}
+
+}  // namespace moe

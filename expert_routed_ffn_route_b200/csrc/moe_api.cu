@@ -38,7 +38,7 @@ moe_status validate(const moe_layer* L) {
   if (L->d > 8192 || L->f > 8192) return MOE_ERR_UNSUPPORTED;
   if (L->E > kMaxE || L->k > kMaxK || L->k > L->E) return MOE_ERR_UNSUPPORTED;
   if ((long long)L->T * L->k > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
-  if (L->path < MOE_PATH_AUTO || L->path > MOE_PATH_TC) return MOE_ERR_INVALID_ARG;
+  if (L->path < MOE_PATH_AUTO || L->path > MOE_PATH_FUSED) return MOE_ERR_INVALID_ARG;
   if (!L->router_w || !aligned(L->router_w, 16)) return MOE_ERR_INVALID_ARG;
   if (L->router_bias && !aligned(L->router_bias, 4)) return MOE_ERR_INVALID_ARG;
   if (!bank_ok(L->routed, L->E, L->d, L->f)) return MOE_ERR_INVALID_ARG;
@@ -60,7 +60,7 @@ WsLayout layout(const moe_layer* L) {
   const size_t n = T * k;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
-  w.status = take(kAlign);
+  w.status = take(sync_bytes(L->d));
   w.logits = take(T * E * sizeof(float));
   w.topk_idx = take(n * sizeof(int32_t));
   w.topk_w = take(n * sizeof(float));
@@ -113,6 +113,8 @@ Plan make_plan(const moe_layer* L, void* ws) {
   p.shared = to_bank(L->shared);
   p.status = reinterpret_cast<int32_t*>(b + w.status);
   p.ticket = reinterpret_cast<int32_t*>(b + w.status + 16);
+  p.gbar = reinterpret_cast<uint32_t*>(b + w.status + 32);
+  p.tile_cnt = reinterpret_cast<int32_t*>(b + w.status + kAlign);
   p.logits = reinterpret_cast<float*>(b + w.logits);
   p.topk_idx = reinterpret_cast<int32_t*>(b + w.topk_idx);
   p.topk_w = reinterpret_cast<float*>(b + w.topk_w);
@@ -160,9 +162,15 @@ bool scales_aligned16(const Bank& b) {
 // dependent launch (their prologue overlaps the tail of the previous kernel).
 // Tensor-core grouped GEMMs for calls with more than 32 tokens (or when asked for).
 bool use_tc(const Plan& p) {
-  if (p.path == MOE_PATH_GEMV) return false;
+  if (p.path == MOE_PATH_GEMV || p.path == MOE_PATH_FUSED) return false;
   if (p.path == MOE_PATH_TC) return true;
   return p.T > 32;
+}
+
+// The single-kernel 1-token layer (decode_fused.cu) when the call allows it.
+bool use_fused(const Plan& p) {
+  if (p.path != MOE_PATH_AUTO && p.path != MOE_PATH_FUSED) return false;
+  return decode_fused_supported(p);
 }
 
 moe_status run_ffn(const Plan& p, cudaStream_t st, void* const* marks, int n_marks) {
@@ -330,6 +338,13 @@ moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, void* out
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> cudaError_t { return record_mark(marks, n_marks, i, st); };
   MOE_TRY(mark(0));
+  if (use_fused(p)) {
+    // one kernel: every stage mark after it
+    MOE_TRY(launch_decode_fused(p, out, p.gbar, p.tile_cnt, st));
+    for (int i = 1; i < MOE_N_MARKS; ++i) MOE_TRY(mark(i));
+    return MOE_OK;
+  }
+  if (p.path == MOE_PATH_FUSED) return MOE_ERR_UNSUPPORTED;
   bool plan_done = false;
   if ((s = run_route(p, st, &plan_done)) != MOE_OK) return s;
   MOE_TRY(mark(1));
@@ -355,6 +370,16 @@ int32_t moe_launches_per_call(const moe_layer* L) {
   p.E = L->E;
   p.k = L->k;
   p.path = L->path;
+  p.d = L->d;
+  p.f = L->f;
+  p.has_shared = L->shared.n_exp;
+  p.routed.fmt = L->routed.fmt;
+  p.shared.fmt = L->shared.fmt;
+  for (int i = 0; i < 3; ++i) {
+    p.routed.s[i] = static_cast<const uint16_t*>(i == 0 ? L->routed.s_gate : i == 1 ? L->routed.s_up : L->routed.s_down);
+    p.shared.s[i] = static_cast<const uint16_t*>(i == 0 ? L->shared.s_gate : i == 1 ? L->shared.s_up : L->shared.s_down);
+  }
+  if (use_fused(p)) return 1;
   const int route = route_fused_supported(p) ? 1 : (2 + (L->T * L->k <= 1024 ? 1 : 3));
   const int ffn = use_tc(p) ? 3 : 2;  // (+ gather/schedule) gate/up, down
   return route + ffn + 1;             // + combine

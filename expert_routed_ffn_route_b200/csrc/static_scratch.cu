@@ -40,8 +40,10 @@ extern "C" moe_status moe_layer_forward_static(const moe_layer* L, const void* x
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_TOO_LARGE;
   void* ws = nullptr;
   if ((s = scratch_address(&ws)) != MOE_OK) return s;
-  // the status word and the routing ticket at the start of the workspace begin at zero
-  if (cudaMemsetAsync(ws, 0, 256, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // the synchronisation block at the start of the workspace (status word, routing ticket,
+  // barrier word, tile counters) begins at zero
+  if (cudaMemsetAsync(ws, 0, moe::sync_bytes(L->d), reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   return moe_layer_forward(L, x, out, nullptr, nullptr, nullptr, nullptr, ws,
                            MOE_STATIC_SCRATCH_BYTES, stream);

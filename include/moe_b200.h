@@ -72,9 +72,13 @@ typedef enum {
 
 typedef enum { MOE_W_BF16 = 16, MOE_W_INT8 = 8, MOE_W_INT4 = 4 } moe_wfmt;
 
-/* Which grouped-FFN kernels run. AUTO picks the tensor-core (tcgen05) grouped GEMMs
- * for large token counts and the split-K GEMV kernels for 1..32-row calls. */
-typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC = 2 } moe_path;
+/* Which kernels run. AUTO picks the single-kernel layer (FUSED) for 1-token calls with
+ * int4 banks when the device fits it, the split-K GEMV kernels for other calls of 1..32
+ * rows, and the tensor-core (tcgen05) grouped GEMMs for larger token counts. FUSED asks for
+ * the single-kernel layer and returns MOE_ERR_UNSUPPORTED from moe_layer_forward when the
+ * call does not fit it; the stage entry points (moe_route ... moe_combine) treat FUSED like
+ * GEMV. */
+typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC = 2, MOE_PATH_FUSED = 3 } moe_path;
 
 /* One expert bank of n_exp experts (the routed bank has n_exp = E; the shared bank has
  * n_exp = 0 or 1). Pointers are device pointers; experts are contiguous, expert e's
@@ -162,7 +166,7 @@ MOE_API moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, v
                                     moe_stream_t stream, void* const* marks, int32_t n_marks);
 
 /* Number of kernels moe_layer_forward enqueues for this descriptor (0 if L is invalid).
- * Host-side only; no CUDA call. */
+ * Host-side only; it may query the current device's multiprocessor count (cached). */
 MOE_API int32_t moe_launches_per_call(const moe_layer* L);
 
 /* Reads the device status word kept in the workspace (synchronises `stream`), writes

@@ -71,16 +71,26 @@ def check_layer(B, dl, L, x_bits, path, sample=None, check_stages=True):
     assert err <= out_tol(ref["out"]), f"max excess {err} > {out_tol(ref['out'])}"
 
     if check_stages:
-        # the four stage entry points give the fused call's result bit for bit
+        # the four stage entry points give the multi-kernel call's result bit for bit (the
+        # single-kernel 1-token layer sums in another order: there, both meet the oracle)
         i2, w2 = B.route(desc, x, ws)
         o2, p2, inv2 = B.permute(desc, i2, ws)
         ya, ys = B.grouped_ffn(desc, x, o2, p2, ws, has_shared=dl.has_shared)
         out3 = B.combine(desc, ya, ys, inv2, w2)
         torch.cuda.synchronize()
-        assert torch.equal(i2, idx) and torch.equal(w2, w)
+        one_kernel = B.launches_per_call(desc) == 1
+        assert torch.equal(i2, idx)
+        if one_kernel:  # logits summed in another order: gates agree to the gate tolerance
+            np.testing.assert_allclose(w2.cpu().numpy(), w.cpu().numpy(), rtol=0, atol=GATE_TOL)
+        else:
+            assert torch.equal(w2, w)
         assert torch.equal(o2, offs) and torch.equal(p2, perm)
         assert np.array_equal(inv2.cpu().numpy(), ref["inv"])
-        assert torch.equal(out3.view(torch.int16), out.view(torch.int16))
+        if one_kernel:
+            got3 = O.widen_bf16(bf16_to_np(out3))[tokens]
+            assert float(output_excess(got3, ref["out"]).max()) <= out_tol(ref["out"])
+        else:
+            assert torch.equal(out3.view(torch.int16), out.view(torch.int16))
     return err
 
 
@@ -155,6 +165,21 @@ def test_full_size_int4(B, int4_bank, name, sample):
     check_layer(B, dl, L, L.x, "auto", sample=sample, check_stages=(cfg.T <= 32))
 
 
+@pytest.mark.parametrize("path,shared", [("gemv", True), ("fused", True), ("fused", False)])
+def test_full_size_decode_paths(B, int4_bank, path, shared):
+    """The decode workload through the multi-kernel GEMV path and the single-kernel path
+    (with and without the shared expert), on several tokens."""
+    cfg = synth.CONFIGS["decode"]
+    routed, sh = int4_bank
+    L = synth.make_layer(cfg, routed=routed, shared=sh)
+    if not shared:
+        L.shared = None
+    dl = B.DeviceLayer(L)
+    for i in range(3):
+        x = L.x if i == 0 else synth.make_hidden(cfg, L.router_w, L.router_bias, stream=f"pool{i}")
+        check_layer(B, dl, L, x, path, check_stages=(i == 0))
+
+
 def test_full_size_long_int8(B):
     cfg = synth.CONFIGS["long"]
     L = synth.make_layer(cfg)
@@ -208,3 +233,64 @@ def test_tc_many_m_tiles(B):
                             seed=13)
     L = synth.make_layer(cfg)
     check_layer(B, B.DeviceLayer(L), L, L.x, "tc", sample=[0, 1, 350, 699])
+
+
+# ------------------------------------------------------------------ single-kernel 1-token layer
+
+def _fused_case(B, cfg):
+    L = synth.make_layer(cfg)
+    dl = B.DeviceLayer(L)
+    assert B.launches_per_call(dl.descriptor(1, "fused")) == 1, "fused path not taken"
+    return L, dl
+
+
+@pytest.mark.parametrize("shared", [1, 0])
+@pytest.mark.parametrize("shape", [(384, 256, 12, 3), (512, 256, 32, 4), (2048, 1024, 64, 8)])
+def test_fused_t1_small(B, shape, shared):
+    d, f, E, k = shape
+    cfg = synth.LayerConfig(f"fused-{d}", T=1, d=d, E=E, k=k, f=f, n_shared=shared, fmt="int4",
+                            seed=31)
+    L, dl = _fused_case(B, cfg)
+    check_layer(B, dl, L, L.x, "fused")
+
+
+def test_fused_t1_many_calls_and_graph(B):
+    """Ten calls in a row on different tokens (the barrier word and the tile counters carry
+    over between calls), then the same calls replayed from a CUDA graph, bit for bit."""
+    cfg = synth.LayerConfig("fused-seq", T=1, d=2048, E=64, k=8, f=1024, fmt="int4", seed=33)
+    L, dl = _fused_case(B, cfg)
+    desc = dl.descriptor(1, "fused")
+    ws = B.alloc_workspace(desc)
+    xs = [synth.make_hidden(cfg, L.router_w, L.router_bias, T=1, stream=f"seq{i}")
+          for i in range(10)]
+    xd = [to_dev_x(x) for x in xs]
+    outs = [B.layer_forward(desc, x, ws) for x in xd]
+    torch.cuda.synchronize()
+    assert B.device_status(desc, ws) == 0
+    for x, o in zip(xs, outs):
+        ref = oracle_run(L, x=x)
+        got = O.widen_bf16(bf16_to_np(o))
+        assert float(output_excess(got, ref["out"]).max()) <= out_tol(ref["out"])
+    st = torch.cuda.Stream()
+    gout = [torch.empty_like(o) for o in outs]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        for x, o in zip(xd, gout):
+            B.layer_forward(desc, x, ws, out=o, stream=st)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert B.device_status(desc, ws) == 0
+    for a, b in zip(outs, gout):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_fused_unsupported_reported(B):
+    cfg = synth.LayerConfig("fused-int8", T=1, d=256, E=8, k=2, f=128, fmt="int8", seed=35)
+    L = synth.make_layer(cfg)
+    dl = B.DeviceLayer(L)
+    desc = dl.descriptor(1, "fused")
+    ws = B.alloc_workspace(desc)
+    with pytest.raises(B.MoeError) as e:
+        B.layer_forward(desc, to_dev_x(L.x), ws)
+    assert e.value.status == -2
