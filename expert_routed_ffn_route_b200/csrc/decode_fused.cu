@@ -50,7 +50,7 @@ constexpr int kDfMaxUnits = 24;
 constexpr int kDfMaxRouter = 8;
 
 #ifdef MOE_TRACE
-__device__ long long g_dftrace[160][16];
+__device__ long long g_dftrace[160][32];
 #define DFT(slot) \
   do { if (threadIdx.x == 0 && blockIdx.x < 160) { unsigned long long _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_dftrace[blockIdx.x][(slot)] = (long long)_t; } } while (0)
 extern "C" __attribute__((visibility("default"))) int moe_dftrace_read(void* dst) {
@@ -69,16 +69,15 @@ struct DfMisc {
   float gate[kMaxK];
   int tile_slot[kDfMaxTiles], tile_rt[kDfMaxTiles];
   int unit_slot[kDfMaxUnits], unit_rt[kDfMaxUnits];
-  int n_tiles, n_units, first_routed, ok, n_combine, armed_tiles, armed_units, armed_h;
-  int combine_rt[kDfMaxUnits];
+  int n_tiles, n_units, n_split, first_routed, ok, armed_tiles, armed_units, armed_h;
 };
 
 // Shared-memory plan of one launch (identical on the host and in every CTA).
 struct DfLayout {
   int grid, n_slots, G, Gf;
-  int tiles_total, tiles_max, units_total, units_max, router_max;
+  int tiles_total, tiles_max, full_per_cta, split_units, units_max, router_max;
   uint32_t tile_bytes, unit_bytes;
-  uint32_t off_router, off_h, off_x, off_xsum, off_red, off_bar, off_misc, total;
+  uint32_t off_router, off_h, off_hsum, off_x, off_xsum, off_cand, off_ybuf, off_red, off_bar, off_misc, total;
 };
 
 __host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int k,
@@ -90,8 +89,13 @@ __host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int
   L.Gf = f / kGroup;
   L.tiles_total = L.n_slots * (f / kDfRows);
   L.tiles_max = (L.tiles_total + grid - 1) / grid;
-  L.units_total = L.n_slots * (d / kDfRows);
-  L.units_max = (L.units_total + grid - 1) / grid;
+  // down units: each CTA owns whole 16-row output tiles (all slots of a tile, combined
+  // locally); the tiles left over are split by slot across CTAs and combined by the CTA
+  // that completes them
+  const int n_rt = d / kDfRows;
+  L.full_per_cta = n_rt / grid;
+  L.split_units = (n_rt - L.full_per_cta * grid) * L.n_slots;
+  L.units_max = L.full_per_cta * L.n_slots + (L.split_units + grid - 1) / grid;
   L.router_max = (E + grid - 1) / grid;
   // gate and up rows (int4) then their bf16 scales
   L.tile_bytes = 2u * kDfRows * (d / 2) + 2u * kDfRows * L.G * 2;
@@ -101,7 +105,9 @@ __host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int
   const uint32_t router_bytes = (uint32_t)L.router_max * d * 2;
   // the h rows of the call (staged after B2) follow the down units
   L.off_h = L.units_max * L.unit_bytes;
-  uint32_t region = max(L.tiles_max * L.tile_bytes, L.off_h + (uint32_t)L.n_slots * f * 2);
+  L.off_hsum = L.off_h + (uint32_t)L.n_slots * f * 2;
+  uint32_t region = max(L.tiles_max * L.tile_bytes, L.off_hsum + 4u * L.n_slots * L.Gf);
+  region = (region + 15) & ~15u;
   if (router_bytes + (has_shared ? L.tile_bytes : 0u) <= region) {
     L.off_router = region - router_bytes;
   } else {
@@ -114,6 +120,24 @@ __host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int
   L.off_xsum = o;
   o += 4u * L.G;
   o = (o + 15) & ~15u;
+  // top-k candidates [ceil(E / 32)][min(k, 32)] (key, index) and their compaction: in the
+  // tile region past buffer 0 when it fits (only the shared tile is live at that time)
+  const uint32_t cand_bytes = 16u * ((E + 31) / 32) * min(k, 32);
+  if (L.tile_bytes + cand_bytes <= region) {
+    L.off_cand = L.tile_bytes;
+  } else {
+    L.off_cand = o;
+    o += cand_bytes;
+  }
+  // y rows of the whole tiles, at the end: past the staged h when it fits
+  const uint32_t ybuf_bytes = 4u * L.full_per_cta * L.n_slots * kDfRows;
+  const uint32_t yb0 = (L.off_hsum + 4u * L.n_slots * L.Gf + 15) & ~15u;
+  if (yb0 + ybuf_bytes <= region) {
+    L.off_ybuf = yb0;
+  } else {
+    L.off_ybuf = o;
+    o += ybuf_bytes;
+  }
   L.off_red = o;
   uint32_t red_gu = (uint32_t)L.tiles_max * 2 * L.G * kDfRows * 4;
   uint32_t red_dn = (uint32_t)L.units_max * L.Gf * kDfRows * 4;
@@ -135,9 +159,15 @@ __host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int
 // 2^31 - (grid - 1) and the others 1, so the top bit flips exactly when the last CTA
 // arrives and the low bits are zero again afterwards. A CTA is through once it sees the
 // top bit differ from the value it found on arrival.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// Arrival: a release (this CTA's writes, ordered before it by the CTA barrier the caller
+// has passed, become visible to every CTA that sees the arrival).
 __device__ __forceinline__ uint32_t gbar_arrive(uint32_t* bar) {
   const uint32_t add = (blockIdx.x == 0) ? (0x80000000u - (gridDim.x - 1)) : 1u;
-  __threadfence();
+  fence_acq_rel_gpu();
   return atomicAdd(bar, add);
 }
 
@@ -150,7 +180,6 @@ __device__ __forceinline__ bool gbar_wait(const uint32_t* bar, uint32_t arrived)
     if (clock64() - t0 > kWaitCycles) return false;
     __nanosleep(32);
   }
-  __threadfence();
   return true;
 }
 
@@ -236,7 +265,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
   uint16_t* s_x = reinterpret_cast<uint16_t*>(smem + L.off_x);
   float* s_xsum = reinterpret_cast<float*>(smem + L.off_xsum);
   float* red = reinterpret_cast<float*>(smem + L.off_red);
-  const uint16_t* s_h = reinterpret_cast<const uint16_t*>(smem + L.off_h);
   uint64_t* bar_router = reinterpret_cast<uint64_t*>(smem + L.off_bar);
   uint64_t* bar_h = bar_router + 1;
   uint64_t* bar_tile = bar_router + 2;
@@ -251,8 +279,17 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
   const int r0 = (int)((long long)E * c / grid), r1 = (int)((long long)E * (c + 1) / grid);
   const int nr = r1 - r0;
   DFT(0);
+#ifdef MOE_TRACE
+  if (tid == 0 && blockIdx.x < 160) g_dftrace[blockIdx.x][26] = clock64();
+#endif
 
   // ---------------------------------------------------------------- prologue
+  const int t0 = (int)((long long)L.tiles_total * c / grid);
+  const int t1 = (int)((long long)L.tiles_total * (c + 1) / grid);
+  // the shared expert's tile of this CTA (at most one: tiles are numbered with the slot
+  // fastest, and slot 0 is the shared expert)
+  const int sh_i = p.has_shared ? (t0 + S - 1) / S * S : t1;
+  const bool has_sh_tile = sh_i < t1;
   if (producer) {
     if (lane == 0) {
       mbar_init(bar_router, 1);
@@ -260,15 +297,15 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       for (int i = 0; i < kDfMaxTiles; ++i) mbar_init(&bar_tile[i], 1);
       for (int i = 0; i < kDfMaxUnits; ++i) mbar_init(&bar_unit[i], 1);
       fence_barrier_init();
-      // first the copies that do not depend on anything: the router rows of this CTA and
-      // its shared-expert tile (at most one: tiles are numbered with the slot fastest)
+      DFTP(1);
+      mi->ok = 1;
+      mi->armed_tiles = has_sh_tile ? 1 : 0;
+      mi->armed_units = 0;
+      mi->armed_h = 0;
+      // the copies that depend on nothing: this CTA's router rows, its shared-expert tile
       const uint32_t rb = (uint32_t)nr * d * 2;
       mbar_arrive_expect_tx(bar_router, rb);
       if (rb) bulk_g2s(smem + L.off_router, p.router_w + (size_t)r0 * d, rb, bar_router);
-      const int t0 = (int)((long long)L.tiles_total * c / grid);
-      const int t1 = (int)((long long)L.tiles_total * (c + 1) / grid);
-      const int sh_i = p.has_shared ? (t0 + S - 1) / S * S : t1;  // first multiple of S >= t0
-      const bool has_sh_tile = sh_i < t1;
       if (has_sh_tile) {
         const size_t row = (size_t)(sh_i / S) * kDfRows;
         const uint32_t wbytes = kDfRows * rowb_up, sbytes = kDfRows * G * 2;
@@ -279,36 +316,57 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         bulk_g2s(smem + 2 * wbytes, p.shared.s[0] + row * G, sbytes, &bar_tile[0]);
         bulk_g2s(smem + 2 * wbytes + sbytes, p.shared.s[1] + row * G, sbytes, &bar_tile[0]);
       }
-      // tile table: the shared tile (if any) first, in buffer 0; routed tiles after it
-      int n = 0;
-      if (has_sh_tile) { mi->tile_slot[0] = 0; mi->tile_rt[0] = sh_i / S; n = 1; }
-      mi->first_routed = n;
-      for (int i = t0; i < t1; ++i)
-        if (i != sh_i) { mi->tile_slot[n] = i % S; mi->tile_rt[n] = i / S; ++n; }
-      mi->n_tiles = n;
-      const int u0 = (int)((long long)L.units_total * c / grid);
-      const int u1 = (int)((long long)L.units_total * (c + 1) / grid);
-      for (int i = u0; i < u1; ++i) { mi->unit_slot[i - u0] = i % S; mi->unit_rt[i - u0] = i / S; }
-      mi->n_units = u1 - u0;
-      mi->ok = 1;
-      mi->armed_tiles = has_sh_tile ? 1 : 0;
-      mi->armed_units = 0;
-      mi->armed_h = 0;
-      if (p.has_shared)
-        for (int i = 0; i < mi->n_units; ++i)
-          if (mi->unit_slot[i] == 0) {
-            const size_t row = (size_t)mi->unit_rt[i] * kDfRows;
-            prefetch_l2(static_cast<const uint8_t*>(p.shared.w[2]) + row * rowb_dn, kDfRows * rowb_dn);
-            prefetch_l2(p.shared.s[2] + row * Gf, kDfRows * Gf * 2);
-          }
+      DFTP(2);
     }
     __syncwarp();
   } else {
     // the activation row (bf16)
     for (int i = tid; i < d / 8; i += kDfCompute)
       reinterpret_cast<uint4*>(s_x)[i] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+    DFT(3);
   }
-  __syncthreads();  // S1: tables, barriers and x
+  __syncthreads();  // S1: barriers initialised, x staged
+
+  if (producer) {
+    // tile and unit tables, one lane an entry: the shared tile (if any) in position 0,
+    // the routed tiles after it in order; units in order
+    const int first_routed = has_sh_tile ? 1 : 0;
+    const int nt = t1 - t0;
+    if (lane < nt) {
+      const int i = t0 + lane;
+      const int pos = (i == sh_i) ? 0 : first_routed + lane - ((has_sh_tile && i > sh_i) ? 1 : 0);
+      mi->tile_slot[pos] = i % S;
+      mi->tile_rt[pos] = i / S;
+    }
+    // units: this CTA's share of the split tiles first, then its whole tiles (slot fastest)
+    const int v0 = (int)((long long)L.split_units * c / grid);
+    const int v1 = (int)((long long)L.split_units * (c + 1) / grid);
+    const int n_split = v1 - v0, n_units = n_split + L.full_per_cta * S;
+    for (int i = lane; i < n_units; i += 32) {
+      int slot, rt;
+      if (i < n_split) {
+        slot = (v0 + i) % S;
+        rt = L.full_per_cta * grid + (v0 + i) / S;
+      } else {
+        slot = (i - n_split) % S;
+        rt = c * L.full_per_cta + (i - n_split) / S;
+      }
+      mi->unit_slot[i] = slot;
+      mi->unit_rt[i] = rt;
+      if (p.has_shared && slot == 0) {  // the shared expert's down rows: into L2 now
+        const size_t row = (size_t)rt * kDfRows;
+        prefetch_l2(static_cast<const uint8_t*>(p.shared.w[2]) + row * rowb_dn, kDfRows * rowb_dn);
+        prefetch_l2(p.shared.s[2] + row * Gf, kDfRows * Gf * 2);
+      }
+    }
+    if (lane == 0) {
+      mi->first_routed = first_routed;
+      mi->n_tiles = nt;
+      mi->n_split = n_split;
+      mi->n_units = n_units;
+    }
+    __syncwarp();
+  }
 
   // ---------------------------------------------------------------- router logits
   if (!producer) {
@@ -322,37 +380,50 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (lane == 0) s_xsum[g] = s;
     }
-    DFT(1);
+    DFT(4);
     if (!mbar_wait(bar_router, 0)) {
       set_status(p.status, DEV_TIMEOUT);
       mi->ok = 0;
     }
-    DFT(2);
+    DFT(5);
     for (int g = warp; g < G; g += kDfWarps) {
       const uint2 xv = *reinterpret_cast<const uint2*>(s_x + g * kGroup + 4 * lane);
       const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
       const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
-      for (int r = 0; r < nr; ++r) {
-        const uint2 wv = *reinterpret_cast<const uint2*>(s_router + (size_t)r * d + g * kGroup + 4 * lane);
-        float s = x0 * __uint_as_float(wv.x << 16);
-        s = fmaf(x1, __uint_as_float(wv.x & 0xffff0000u), s);
-        s = fmaf(x2, __uint_as_float(wv.y << 16), s);
-        s = fmaf(x3, __uint_as_float(wv.y & 0xffff0000u), s);
+      float s[kDfMaxRouter];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) red[r * G + g] = s;
+      for (int r = 0; r < kDfMaxRouter; ++r) {
+        s[r] = 0.f;
+        if (r < nr) {
+          const uint2 wv = *reinterpret_cast<const uint2*>(s_router + (size_t)r * d + g * kGroup + 4 * lane);
+          s[r] = x0 * __uint_as_float(wv.x << 16);
+          s[r] = fmaf(x1, __uint_as_float(wv.x & 0xffff0000u), s[r]);
+          s[r] = fmaf(x2, __uint_as_float(wv.y << 16), s[r]);
+          s[r] = fmaf(x3, __uint_as_float(wv.y & 0xffff0000u), s[r]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int r = 0; r < kDfMaxRouter; ++r) s[r] += __shfl_xor_sync(0xffffffffu, s[r], o);
+      if (lane == 0) {
+#pragma unroll
+        for (int r = 0; r < kDfMaxRouter; ++r)
+          if (r < nr) red[r * G + g] = s[r];
       }
     }
     named_bar_sync(1, kDfCompute);
-    if (tid < nr) {
+    for (int r = warp; r < nr; r += kDfWarps) {  // a warp a row: fixed-order tree over groups
       float s = 0.f;
-      for (int g = 0; g < G; ++g) s += red[tid * G + g];
-      const int e = r0 + tid;
-      p.logits[e] = s + (p.router_bias ? p.router_bias[e] : 0.f);
+      for (int g = lane; g < G; g += 32) s += red[r * G + g];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const int e = r0 + r;
+      if (lane == 0) p.logits[e] = s + (p.router_bias ? p.router_bias[e] : 0.f);
     }
+    DFT(6);
   }
   __syncthreads();  // S2: this CTA's logits are written
-  DFT(3);
 
   // Items (tile position b, matrix m, group g), warp w takes every kDfWarps-th item of a
   // tile range; partials land in red[b][m][g][16] (rows of the tile), scaled and corrected.
@@ -367,7 +438,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         return;
       }
 #ifdef MOE_TRACE
-      if (warp == 0 && b == mi->first_routed) DFT(8);
+      if (warp == 0 && b == mi->first_routed) DFT(13);
 #endif
       const uint8_t* tile = smem + (size_t)b * L.tile_bytes;
       const uint16_t* scales = reinterpret_cast<const uint16_t*>(tile + 2 * kDfRows * rowb_up);
@@ -396,42 +467,137 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
   if (producer) {
     if (lane == 0) {
       s_arrived = gbar_arrive(gbar);
+      DFTP(7);
       if (mi->ok && !gbar_wait(gbar, s_arrived)) {
         set_status(p.status, DEV_TIMEOUT);
         mi->ok = 0;
       }
-      DFTP(4);
+      DFTP(8);
     }
     __syncwarp();  // the warp reaches the CTA barrier converged
   } else if (mi->ok) {
     gate_up_items(0, mi->first_routed);  // the shared tile, while B1 settles
   }
   __syncthreads();  // S3
-  DFT(5);
 
   // ---------------------------------------------------------------- top-k (every CTA)
-  if (mi->ok && warp == 0) {
-    int e;
-    uint32_t key;
-    DFT(7);
-    warp_topk(p.logits, E, k, lane, &e, &key);
-    DFT(12);
-    const uint32_t top = __shfl_sync(0xffffffffu, key, 0);
-    const float gte = warp_topk_gate(key, top, k, lane);
-    if (lane < k) {
-      mi->sel[lane] = e;
-      mi->gate[lane] = gte;
+  // "a beats b": a larger logit, or an equal logit and a lower expert index; the k picks
+  // are the experts that fewer than k others beat, in that order. Level 1: warp w ranks
+  // each chunk of 32 consecutive experts (one per lane, 32 shuffles) and lists the chunk's
+  // first kk = min(k, 32) in rank order. Level 2: each listed candidate among the first k
+  // of its list counts, by binary search, how many entries of every other list beat it;
+  // the sum is its overall rank. Gates: softmax over the picks, summed by a fixed tree.
+  if (mi->ok && !producer) {
+    const int n_chunks = (E + 31) / 32;
+    const int kk = min(k, 32);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(smem + L.off_cand);  // [chunk][kk] key, idx
+    DFT(9);
+    for (int ch = warp; ch < n_chunks; ch += kDfWarps) {
+      const int e = ch * 32 + lane;
+      const uint32_t key = (e < E) ? order_key(__ldcg(p.logits + e)) : 0u;
+      int rank = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const uint32_t kj = __shfl_sync(0xffffffffu, key, j);
+        rank += (kj > key) || (kj == key && j < lane);
+      }
+      if (rank < kk) {
+        cand[2 * (ch * kk + rank)] = key;
+        cand[2 * (ch * kk + rank) + 1] = (e < E) ? (uint32_t)e : 0xffffffffu;
+      }
+    }
+    named_bar_sync(1, kDfCompute);
+    DFT(10);
+    // level 2 (warp 0): the k-th best chunk head bounds the picks from below (the k heads at
+    // least as good beat anything it beats), so only candidates it does not beat remain;
+    // they are ranked among themselves with shuffles (their overall rank: whatever beats a
+    // remaining candidate remains too). More than 32 remaining (heavy ties): a table scan.
+    if (warp == 0) {
+      auto beats = [](uint32_t ka, uint32_t ia, uint32_t kb, uint32_t ib) {
+        return ka > kb || (ka == kb && ia < ib);
+      };
+      const int n_cand = n_chunks * kk;
+      uint32_t tk = 0u, ti = 0xffffffffu;  // the threshold: beats nothing valid by default
+      if (n_chunks >= k) {
+        const uint32_t hk = (lane < n_chunks) ? cand[2 * (lane * kk)] : 0u;
+        const uint32_t hx = (lane < n_chunks) ? cand[2 * (lane * kk) + 1] : 0xffffffffu;
+        int hr = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const uint32_t kj = __shfl_sync(0xffffffffu, hk, j), xj = __shfl_sync(0xffffffffu, hx, j);
+          hr += (j < n_chunks) && beats(kj, xj, hk, hx);
+        }
+        const unsigned at = __ballot_sync(0xffffffffu, lane < n_chunks && hr == k - 1);
+        const int tl = __ffs(at) - 1;
+        tk = __shfl_sync(0xffffffffu, hk, tl);
+        ti = __shfl_sync(0xffffffffu, hx, tl);
+      }
+      // compact the candidates the threshold does not beat (in table order)
+      uint32_t* keep = cand + 2 * n_cand;  // room for n_cand entries after the table
+      int n_keep = 0;
+      for (int t0 = 0; t0 < n_cand; t0 += 32) {
+        const int t = t0 + lane;
+        uint32_t ck = 0u, cx = 0xffffffffu;
+        if (t < n_cand) {
+          ck = cand[2 * t];
+          cx = cand[2 * t + 1];
+        }
+        const bool kp = (t < n_cand) && ck != 0u && !beats(tk, ti, ck, cx);
+        const unsigned bal = __ballot_sync(0xffffffffu, kp);
+        if (kp) {
+          const int at = n_keep + __popc(bal & ((1u << lane) - 1u));
+          keep[2 * at] = ck;
+          keep[2 * at + 1] = cx;
+        }
+        n_keep += __popc(bal);
+      }
+      __syncwarp();
+      if (n_keep <= 32) {
+        const uint32_t ck = (lane < n_keep) ? keep[2 * lane] : 0u;
+        const uint32_t cx = (lane < n_keep) ? keep[2 * lane + 1] : 0xffffffffu;
+        int rank = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const uint32_t kj = __shfl_sync(0xffffffffu, ck, j), xj = __shfl_sync(0xffffffffu, cx, j);
+          rank += (j < n_keep) && beats(kj, xj, ck, cx);
+        }
+        if (lane < n_keep && rank < k) {
+          mi->sel[rank] = (int)cx;
+          reinterpret_cast<uint32_t*>(mi->gate)[rank] = ck;  // key for now, gate below
+        }
+      } else {
+        for (int t = lane; t < n_keep; t += 32) {
+          const uint32_t ck = keep[2 * t], cx = keep[2 * t + 1];
+          int rank = 0;
+          for (int j = 0; j < n_keep; ++j) rank += beats(keep[2 * j], keep[2 * j + 1], ck, cx);
+          if (rank < k) {
+            mi->sel[rank] = (int)cx;
+            reinterpret_cast<uint32_t*>(mi->gate)[rank] = ck;
+          }
+        }
+      }
+    }
+    named_bar_sync(1, kDfCompute);
+    if (warp == 0) {
+      const uint32_t my_key = (lane < k) ? reinterpret_cast<const uint32_t*>(mi->gate)[lane] : 0u;
+      const uint32_t top = __shfl_sync(0xffffffffu, my_key, 0);
+      const float z = (lane < k) ? expf(key_value(my_key) - key_value(top)) : 0.f;
+      float tot = z;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      __syncwarp();
+      if (lane < k) mi->gate[lane] = z / tot;
+      DFT(11);
     }
   }
   __syncthreads();  // S4: the routing decision
-  DFT(6);
   const bool ok1 = mi->ok;
 
   // ---------------------------------------------------------------- gate/up tiles
   if (producer) {
     if (ok1) {
-      // routed tiles, one lane a tile (the router rows they overwrite are consumed)
-      fence_proxy_async();
+      // routed tiles, one lane a tile (the router rows they overwrite were consumed before
+      // the CTA barrier above)
       const int b = mi->first_routed + lane;
       if (b < mi->n_tiles) {
         const uint32_t wbytes = kDfRows * rowb_up, sbytes = kDfRows * G * 2;
@@ -446,6 +612,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         bulk_g2s(dst + 2 * wbytes + sbytes, p.routed.s[1] + row * G, sbytes, &bar_tile[b]);
       }
       if (lane == 0) mi->armed_tiles = mi->n_tiles;
+      if (lane == 0) DFTP(12);
       __syncwarp();
       // the routed down rows this CTA will need, into L2 behind the gate/up requests
       for (int i = lane; i < mi->n_units; i += 32) {
@@ -475,34 +642,14 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       }
     }
     gate_up_items(mi->first_routed, mi->n_tiles);
-    DFT(9);
+    DFT(14);
   }
-  __syncthreads();  // S5: every gate/up product of this CTA is in red
-  DFT(10);
+  __syncthreads();  // S5: every gate/up product of this CTA is in red; tile buffers are free
 
-  // h rows of this CTA's tiles: fixed-order sums over the K groups, SwiGLU, one rounding
-  if (ok1 && !producer) {
-    for (int i = tid; i < mi->n_tiles * kDfRows; i += kDfCompute) {
-      const int b = i / kDfRows, r = i % kDfRows;
-      const float* rg = red + (size_t)(b * 2) * G * kDfRows + r;
-      const float* ru = rg + (size_t)G * kDfRows;
-      float gs = 0.f, us = 0.f;
-      for (int g = 0; g < G; ++g) {
-        gs += rg[g * kDfRows];
-        us += ru[g * kDfRows];
-      }
-      const float hv = gs / (1.f + expf(-gs)) * us;
-      p.h[(size_t)mi->tile_slot[b] * f + (size_t)mi->tile_rt[b] * kDfRows + r] = f32_to_bf16_rn(hv);
-    }
-  }
-  __syncthreads();  // S6: h of this CTA written; the tile buffers are free
-  DFT(11);
-
-  // ---------------------------------------------------------------- B2
   if (producer) {
     if (ok1) {
-      // down units into the freed tile buffers (from L2 when the prefetch has landed)
-      fence_proxy_async();
+      // down units into the freed tile buffers (from L2 when the prefetch has landed), one
+      // lane a unit, while the compute warps finish h
       for (int i = lane; i < mi->n_units; i += 32) {
         const int slot = mi->unit_slot[i];
         const bool sh = p.has_shared && slot == 0;
@@ -516,14 +663,38 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         bulk_g2s(dst + wbytes, bk.s[2] + row * Gf, sbytes, &bar_unit[i]);
       }
       if (lane == 0) mi->armed_units = mi->n_units;
+      if (lane == 0) DFTP(16);
     }
+    __syncwarp();
+  } else if (ok1) {
+    // h rows of this CTA's tiles: fixed-order sums over the K groups, SwiGLU, one rounding
+    for (int i = tid; i < mi->n_tiles * kDfRows; i += kDfCompute) {
+      const int b = i / kDfRows, r = i % kDfRows;
+      const float* rg = red + (size_t)(b * 2) * G * kDfRows + r;
+      const float* ru = rg + (size_t)G * kDfRows;
+      float gs = 0.f, us = 0.f;
+      for (int g = 0; g < G; ++g) {
+        gs += rg[g * kDfRows];
+        us += ru[g * kDfRows];
+      }
+      const float hv = gs / (1.f + expf(-gs)) * us;
+      p.h[(size_t)mi->tile_slot[b] * f + (size_t)mi->tile_rt[b] * kDfRows + r] = f32_to_bf16_rn(hv);
+    }
+    DFT(15);
+  }
+  __syncthreads();  // S6: h of this CTA written
+
+  // ---------------------------------------------------------------- B2
+  if (producer) {
     // every CTA arrives at every barrier, failed or not, so the word stays consistent
     if (lane == 0) {
       s_arrived = gbar_arrive(gbar);
+      DFTP(17);
       if (ok1 && !gbar_wait(gbar, s_arrived)) {
         set_status(p.status, DEV_TIMEOUT);
         mi->ok = 0;
       }
+      DFTP(18);
       if (mi->ok) {  // every h row of the call, into shared memory in one request
         mbar_arrive_expect_tx(bar_h, (uint32_t)S * f * 2);
         mi->armed_h = 1;
@@ -535,93 +706,170 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     if (mi->ok)
       for (int s = lane; s < S; s += 32)
         bulk_g2s(smem + L.off_h + (size_t)s * f * 2, p.h + (size_t)s * f, f * 2, bar_h);
+    if (lane == 0) DFTP(19);
     __syncwarp();
   }
   __syncthreads();  // S7: the B2 verdict
   const bool ok2 = mi->ok;
 
   // ---------------------------------------------------------------- down units
-  if (ok2 && !producer) {
-    if (!warp_wait(bar_h)) {
-      if (lane == 0) set_status(p.status, DEV_TIMEOUT);
-    } else {
-      uint32_t xb[16];
-      for (int u = 0; u < mi->n_units; ++u) {
-        const int slot = mi->unit_slot[u];
-        const uint8_t* unit = smem + (size_t)u * L.unit_bytes;
-        const uint16_t* scales = reinterpret_cast<const uint16_t*>(unit + kDfRows * rowb_dn);
-        // items (u, g) in one flat order over the CTA's units: warp w takes u * Gf + g = w mod W
-        const int first = ((warp - u * Gf) % kDfWarps + kDfWarps) % kDfWarps;
-        if (first >= Gf) continue;
-        if (!warp_wait(&bar_unit[u])) {
-          if (lane == 0) set_status(p.status, DEV_TIMEOUT);
-          break;
+  // Compute warps: h to fragment order (+ group sums); pass A, the units of split tiles, and
+  // their y rows to the workspace; then (the producer meanwhile posts the split-tile
+  // arrivals and combines the split tiles it completes) pass B, the whole tiles, combined
+  // locally. Both combines sum the gates in rank order, then the shared term, in fp32.
+  uint16_t* hw = reinterpret_cast<uint16_t*>(smem + L.off_h);
+  float* s_hsum = reinterpret_cast<float*>(smem + L.off_hsum);
+  auto down_items = [&](int u_begin, int u_end) {
+    uint32_t xb[16];
+    for (int u = u_begin; u < u_end; ++u) {
+      const int slot = mi->unit_slot[u];
+      const uint8_t* unit = smem + (size_t)u * L.unit_bytes;
+      const uint16_t* scales = reinterpret_cast<const uint16_t*>(unit + kDfRows * rowb_dn);
+      // items (u, g) in u-major order from u_begin: warp w takes every kDfWarps-th
+      const int first = ((warp - (u - u_begin) * Gf) % kDfWarps + kDfWarps) % kDfWarps;
+      if (first >= Gf) continue;
+      if (!warp_wait(&bar_unit[u])) {
+        if (lane == 0) set_status(p.status, DEV_TIMEOUT);
+        return;
+      }
+      for (int g = first; g < Gf; g += kDfWarps) {
+        const uint16_t* hrow = hw + (size_t)slot * f + g * kGroup + 32 * q;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (grp == 0) v = *reinterpret_cast<const uint4*>(hrow + 8 * i);
+          xb[4 * i + 0] = v.x;
+          xb[4 * i + 1] = v.y;
+          xb[4 * i + 2] = v.z;
+          xb[4 * i + 3] = v.w;
         }
-        for (int g = first; g < Gf; g += kDfWarps) {
-          float hs = t1_load_act<false>(s_h + (size_t)slot * f, g, q, grp == 0, xb);
-          hs = __shfl_sync(0xffffffffu, hs, 0);
-          float ra, rb;
-          t1_group(unit, rowb_dn, g, grp, q, xb, ra, rb);
-          if (q == 0) {
-            const uint16_t* sc = scales + g;
-            const float corr = 136.f * hs;
-            float* dst = red + ((size_t)u * Gf + g) * kDfRows;
-            dst[grp] = bf16_to_f32(sc[grp * Gf]) * (ra - corr);
-            dst[grp + 8] = bf16_to_f32(sc[(grp + 8) * Gf]) * (rb - corr);
-          }
+        float ra, rb;
+        t1_group(unit, rowb_dn, g, grp, q, xb, ra, rb);
+        if (q == 0) {
+          const uint16_t* sc = scales + g;
+          const float corr = 136.f * s_hsum[slot * Gf + g];
+          float* dst = red + ((size_t)u * Gf + g) * kDfRows;
+          dst[grp] = bf16_to_f32(sc[grp * Gf]) * (ra - corr);
+          dst[grp + 8] = bf16_to_f32(sc[(grp + 8) * Gf]) * (rb - corr);
         }
       }
     }
-  }
-  __syncthreads();  // S8
-  DFT(13);
-  if (ok2 && !producer) {
-    for (int i = tid; i < mi->n_units * kDfRows; i += kDfCompute) {
-      const int u = i / kDfRows, r = i % kDfRows;
-      const float* src = red + (size_t)u * Gf * kDfRows + r;
-      float y = 0.f;
-      for (int g = 0; g < Gf; ++g) y += src[g * kDfRows];
-      const int slot = mi->unit_slot[u];
-      const size_t n = (size_t)mi->unit_rt[u] * kDfRows + r;
-      if (p.has_shared && slot == 0) p.y_shared[n] = y;
-      else p.y_assign[(size_t)(slot - p.has_shared) * d + n] = y;
-    }
-  }
-  __syncthreads();  // S9: this CTA's y values written
+  };
+  // y of unit u, row r: the fixed-order sum of its K-group partials
+  auto unit_y = [&](int u, int r) {
+    const float* src_r = red + (size_t)u * Gf * kDfRows + r;
+    float y = 0.f;
+    for (int g = 0; g < Gf; ++g) y += src_r[g * kDfRows];
+    return y;
+  };
+
   if (producer) {
-    // Arrivals per output tile (one lane a tile; the CTA's units are consecutive, so each
-    // tile's units form one run). The CTA that completes a tile combines it.
-    const int nu = mi->n_units;
-    const int first_rt = nu ? mi->unit_rt[0] : 0;
+    named_bar_sync(2, kDfThreads);  // the split-tile y rows of this CTA are written
+    // Arrivals on the split tiles, one lane a tile (this CTA's split units are consecutive).
+    // Every CTA posts its arrivals, failed or not, so the counters return to zero.
+    const int ns = mi->n_split;
+    const int first_rt = ns ? mi->unit_rt[0] : 0;
     const int rt = first_rt + lane;
     int n = 0;
-    for (int i = 0; i < nu; ++i) n += (mi->unit_rt[i] == rt);
+    for (int i = 0; i < ns; ++i) n += (mi->unit_rt[i] == rt);
     bool mine = false;
     if (n > 0) {
-      __threadfence();
+      fence_acq_rel_gpu();
       const int old = atomicAdd(&tile_cnt[rt], n);
       if (old + n == S) {
         tile_cnt[rt] = 0;  // every unit of the tile has arrived: ready for the next call
-        mine = ok2;
-        __threadfence();
+        mine = ok2 && mi->ok;
+        fence_acq_rel_gpu();
       }
     }
-    const unsigned m = __ballot_sync(0xffffffffu, mine);
-    if (mine) mi->combine_rt[__popc(m & ((1u << lane) - 1u))] = rt;
-    if (lane == 0) mi->n_combine = __popc(m);
-  }
-  __syncthreads();  // S10
-  DFT(14);
-  if (ok2 && !producer) {
-    for (int i = tid; i < mi->n_combine * kDfRows; i += kDfCompute) {
-      const size_t n = (size_t)mi->combine_rt[i / kDfRows] * kDfRows + i % kDfRows;
-      float acc = 0.f;
-      for (int j = 0; j < k; ++j) acc = fmaf(mi->gate[j], __ldcg(p.y_assign + (size_t)j * d + n), acc);
-      if (p.has_shared) acc += __ldcg(p.y_shared + n);
-      out[n] = f32_to_bf16_rn(acc);
+    unsigned m = __ballot_sync(0xffffffffu, mine);
+    while (m) {  // combine the split tiles this CTA completed
+      const int src_lane = __ffs(m) - 1;
+      m &= m - 1;
+      const int crt = __shfl_sync(0xffffffffu, rt, src_lane);
+      if (lane < kDfRows) {
+        const size_t nn = (size_t)crt * kDfRows + lane;
+        float acc = 0.f;
+        for (int j = 0; j < k; ++j)
+          acc = fmaf(mi->gate[j], __ldcg(p.y_assign + (size_t)j * d + nn), acc);
+        if (p.has_shared) acc += __ldcg(p.y_shared + nn);
+        out[nn] = f32_to_bf16_rn(acc);
+      }
+    }
+    if (lane == 0) DFTP(24);
+    __syncwarp();
+  } else {
+    bool ready = false;
+    if (ok2) {
+      ready = warp_wait(bar_h);
+      if (!ready && lane == 0) set_status(p.status, DEV_TIMEOUT);
+      DFT(20);
+      // h rows -> fragment order in place, and their per-group sums (a half-warp a group:
+      // each lane one 8-value chunk, then a fixed tree over the 16 chunks)
+      const int n_groups = S * Gf;
+      for (int gi = 2 * warp + (lane >> 4); gi < n_groups && ready; gi += 2 * kDfWarps) {
+        uint4* chunk = reinterpret_cast<uint4*>(hw + (size_t)gi * kGroup) + (lane & 15);
+        uint4 v = *chunk;
+        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          s += __uint_as_float(vv[j] << 16);
+          s += __uint_as_float(vv[j] & 0xffff0000u);
+        }
+        permute_chunk<4>(v);
+        *chunk = v;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if ((lane & 15) == 0) s_hsum[gi] = s;
+      }
+    }
+    named_bar_sync(1, kDfCompute);
+    if (ok2 && ready) down_items(0, mi->n_split);  // pass A
+    named_bar_sync(1, kDfCompute);
+    if (ok2) {
+      for (int i = tid; i < mi->n_split * kDfRows; i += kDfCompute) {
+        const int u = i / kDfRows, r = i % kDfRows;
+        const float y = unit_y(u, r);
+        const int slot = mi->unit_slot[u];
+        const size_t n = (size_t)mi->unit_rt[u] * kDfRows + r;
+        if (p.has_shared && slot == 0) p.y_shared[n] = y;
+        else p.y_assign[(size_t)(slot - p.has_shared) * d + n] = y;
+      }
+    }
+    named_bar_sync(2, kDfThreads);
+    DFT(21);
+    if (ok2 && ready) down_items(mi->n_split, mi->n_units);  // pass B
+    DFT(22);
+    named_bar_sync(1, kDfCompute);
+    if (ok2) {
+      // y of every whole-tile unit row into red's first row of the unit (in place: a row's
+      // partials are read before any thread writes that row's slot 0)
+      float* ybuf = reinterpret_cast<float*>(smem + L.off_ybuf);  // [units][16]
+      for (int i = tid; i < (mi->n_units - mi->n_split) * kDfRows; i += kDfCompute) {
+        const int u = mi->n_split + i / kDfRows, r = i % kDfRows;
+        ybuf[i] = unit_y(u, r);
+      }
+    }
+    named_bar_sync(1, kDfCompute);
+    if (ok2) {
+      const float* ybuf = reinterpret_cast<const float*>(smem + L.off_ybuf);
+      const int n_full = (mi->n_units - mi->n_split) / S;
+      for (int i = tid; i < n_full * kDfRows; i += kDfCompute) {
+        const int t = i / kDfRows, r = i % kDfRows;
+        const float* yt = ybuf + (size_t)t * S * kDfRows + r;  // slot s at yt[s * 16]
+        float acc = 0.f;
+        for (int j = 0; j < k; ++j) acc = fmaf(mi->gate[j], yt[(p.has_shared + j) * kDfRows], acc);
+        if (p.has_shared) acc += yt[0];
+        out[(size_t)mi->unit_rt[mi->n_split + t * S] * kDfRows + r] = f32_to_bf16_rn(acc);
+      }
+      DFT(25);
     }
   }
-  DFT(15);
+  __syncthreads();
+#ifdef MOE_TRACE
+  if (tid == 0 && blockIdx.x < 160) g_dftrace[blockIdx.x][27] = clock64();
+#endif
 
   // ---------------------------------------------------------------- drain
   // No copy may land after the CTA ends: wait (boundedly) for every one that was issued.
