@@ -403,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic(cfg.name, "decode_fused" if fused else
-                                                 ("tc_grouped" if cfg.T > 32 else "gemv_tma")),
+                                                 ("tc_grouped" if cfg.T >= 16 else "gemv_tma")),
                      "avg_launch_ms": gu_avg_ms,
                      "layer_frac": float(np.mean(layer_bytes)) / (ms_per_step * 1e-3) / 1e9 / peak},
         "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",

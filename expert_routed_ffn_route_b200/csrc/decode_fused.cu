@@ -512,6 +512,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     // least as good beat anything it beats), so only candidates it does not beat remain;
     // they are ranked among themselves with shuffles (their overall rank: whatever beats a
     // remaining candidate remains too). More than 32 remaining (heavy ties): a table scan.
+#ifdef MOE_TRACE
+    for (int rep = 0; rep < 2; ++rep) {
+      if (rep == 1) DFT(23);
+#endif
     if (warp == 0) {
       auto beats = [](uint32_t ka, uint32_t ia, uint32_t kb, uint32_t ib) {
         return ka > kb || (ka == kb && ia < ib);
@@ -577,6 +581,9 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         }
       }
     }
+#ifdef MOE_TRACE
+    }
+#endif
     named_bar_sync(1, kDfCompute);
     if (warp == 0) {
       const uint32_t my_key = (lane < k) ? reinterpret_cast<const uint32_t*>(mi->gate)[lane] : 0u;
@@ -596,20 +603,28 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
   // ---------------------------------------------------------------- gate/up tiles
   if (producer) {
     if (ok1) {
-      // routed tiles, one lane a tile (the router rows they overwrite were consumed before
-      // the CTA barrier above)
-      const int b = mi->first_routed + lane;
-      if (b < mi->n_tiles) {
+      // routed tiles, six copies each (gate and up in halves of 8 rows, then their scales),
+      // one lane a copy; every tile's byte count is posted before any of its copies. The
+      // router rows they overwrite were consumed before the CTA barrier above.
+      const int n_routed = mi->n_tiles - mi->first_routed;
+      if (lane < n_routed) mbar_arrive_expect_tx(&bar_tile[mi->first_routed + lane], L.tile_bytes);
+      __syncwarp();
+      for (int i = lane; i < 6 * n_routed; i += 32) {
+        const int b = mi->first_routed + i / 6, part = i % 6;
         const uint32_t wbytes = kDfRows * rowb_up, sbytes = kDfRows * G * 2;
         const int j = mi->tile_slot[b] - p.has_shared;
         const size_t row = (size_t)mi->sel[j] * f + (size_t)mi->tile_rt[b] * kDfRows;
         uint8_t* dst = smem + (size_t)b * L.tile_bytes;
-        mbar_arrive_expect_tx(&bar_tile[b], L.tile_bytes);
-        bulk_g2s(dst, static_cast<const uint8_t*>(p.routed.w[0]) + row * rowb_up, wbytes, &bar_tile[b]);
-        bulk_g2s(dst + wbytes, static_cast<const uint8_t*>(p.routed.w[1]) + row * rowb_up, wbytes,
-                 &bar_tile[b]);
-        bulk_g2s(dst + 2 * wbytes, p.routed.s[0] + row * G, sbytes, &bar_tile[b]);
-        bulk_g2s(dst + 2 * wbytes + sbytes, p.routed.s[1] + row * G, sbytes, &bar_tile[b]);
+        if (part < 4) {
+          const int m = part >> 1, half = part & 1;
+          const uint32_t hb = wbytes / 2;
+          bulk_g2s(dst + m * wbytes + half * hb,
+                   static_cast<const uint8_t*>(p.routed.w[m]) + row * rowb_up + half * hb, hb,
+                   &bar_tile[b]);
+        } else {
+          const int m = part - 4;
+          bulk_g2s(dst + 2 * wbytes + m * sbytes, p.routed.s[m] + row * G, sbytes, &bar_tile[b]);
+        }
       }
       if (lane == 0) mi->armed_tiles = mi->n_tiles;
       if (lane == 0) DFTP(12);

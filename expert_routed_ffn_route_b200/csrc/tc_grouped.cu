@@ -10,16 +10,18 @@
 // walked in chunks of 64. D lives in TMEM (lane = weight row, column = token).
 //
 // One persistent CTA per SM, warp roles:
-//   warp 0      TMA producer: raw weight tiles [128 rows x 64 K] (int4/int8/bf16, no
-//               swizzle) and activation tiles [N rows x 64 K] bf16 (128-byte swizzle)
+//   warp 0      TMA producer of the raw weight stages [128 rows x 128 bytes] (int4/int8/
+//               bf16, 128-byte swizzle) and each unit's group scales
 //   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16, fp32
 //               accumulate; for gate/up warp 14 issues the up-projection MMAs in parallel
 //               (separate accumulator), which halves the instructions one thread issues
-//   warps 2-9   dequantisers: two threads per weight row, W = fp16(q * s) written straight
-//               from registers into TMEM (tcgen05.st), where the MMA reads its A operand;
+//   warps 2-9   dequantisers, two groups of four taking alternate chunks: W = fp16(q * s)
+//               written straight from registers into TMEM (tcgen05.st), where the MMA
+//               reads its A operand;
 //               shared memory then carries only the raw weights and the activations
 //   warps 10-13 epilogue: tcgen05.ld of their 32 TMEM lanes; gate/up: h = silu(g) * u ->
 //               fp16 rows; down: fp32 rows
+//   warp 15     TMA producer of the activation tiles (warp 0 streams the weights)
 // Operands are fp16 (kind::f16, fp32 accumulate): the activations (bf16 inputs) convert to
 // fp16 exactly in fp16's range, and q * s rounds once with an 11-bit significand, eight
 // times finer than bf16. Activations and h outside fp16's range set a device status flag.
@@ -61,8 +63,9 @@ extern "C" __attribute__((visibility("default"))) int moe_tct_read(void* dst) {
 #define TCC(c, ev) do {} while (0)
 #endif
 
-constexpr int kTcThreads = 480;  // 15 warps
+constexpr int kTcThreads = 512;  // 16 warps
 constexpr int kDqWarps = 8;       // dequantisers (two threads per weight row)
+constexpr int kIssuers = 2;       // MMA issuing threads (warps 1 and 14)
 constexpr int kTcBK = 64;      // K per chunk (one 128-byte swizzle span of bf16)
 constexpr int kTcM = 128;      // weight rows per tile
 constexpr int kTcNMax = 64;    // token rows per tile
@@ -76,17 +79,22 @@ struct TcMaps {
 
 template <int FMT, bool GATE_UP> struct TcCfg {
   static constexpr int NM = GATE_UP ? 2 : 1;
-  static constexpr int RAW_ROW = kTcBK * FMT / 8;    // raw bytes of one row per chunk
-  static constexpr int RAW = kTcM * RAW_ROW;         // one raw matrix chunk
+  // A weight stage is 128 bytes of each of 128 rows (one 128-byte swizzle span: full L2
+  // lines per row and conflict-free reads), i.e. KW = 256 / 128 / 64 K values for int4 /
+  // int8 / bf16, walked by the dequantisers in SUB chunks of kTcBK.
+  static constexpr int RAW_ROW = 128;                // raw bytes of one row per stage
+  static constexpr int KW = RAW_ROW * 8 / FMT;       // K values per stage
+  static constexpr int SUB = KW / kTcBK;             // kTcBK chunks per stage
+  static constexpr int RAW = kTcM * RAW_ROW;         // one raw matrix stage
   static constexpr int XB = kTcNMax * kTcBK * 2;     // activation stage bytes
   // Ring depths: the weight ring is deep (HBM latency) and is released by the dequantisers
   // as soon as they have read it; the activation ring (mostly L2 hits) by the tensor core.
   static constexpr int WB = NM * RAW;                // weight stage bytes
   static constexpr int W_BUDGET = (GATE_UP ? 128 : 96) * 1024;
   static constexpr int NW = W_BUDGET / WB > 16 ? 16 : W_BUDGET / WB;
-  static constexpr int NX = 6;
+  static constexpr int NX = GATE_UP ? 4 : 6;         // activation stages (= A stages)
   static constexpr int A_COLS = NM * (kTcBK / 2);    // TMEM columns of one A stage
-  static constexpr int NA = GATE_UP ? 4 : 6;         // A stages in TMEM
+  static constexpr int NA = NX;                      // A stages in TMEM
   static constexpr int A_COL0 = 256;
   static_assert(A_COL0 + NA * A_COLS <= 512, "TMEM budget");
   // layout (1024-byte aligned pieces first)
@@ -165,6 +173,16 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// The same, accumulating into D unconditionally (no per-instruction predicate set-up).
+__device__ __forceinline__ void umma_f16_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc)
+      : "memory");
+}
+
 // 16 consecutive 32-bit columns of this thread's TMEM lane <- registers.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -173,6 +191,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane <- registers (one instruction:
+// tcgen05 instructions cost each issuing thread about a hundred cycles or more).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
 
@@ -313,16 +345,21 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
 
 // ------------------------------------------------------------------ dequantisation
 
-// Half `half` (K values 32*half .. 32*half+31) of a raw chunk row (64 K values of one
-// weight row) -> 32 fp16 = W * s in K order, two per register.
+// Half `half` (K values 32*half .. 32*half+31) of chunk `s` (K values 64*s .. 64*s+63 of the
+// stage) of one weight row -> 32 fp16 = W * s in K order, two per register. The row is one
+// 128-byte line of a stage written by the TMA with 128-byte swizzling: its 16-byte piece j
+// sits at piece j ^ sw7 (sw7 = the row index mod 8).
 template <int FMT>
-__device__ __forceinline__ void dequant_half_row(const uint8_t* raw_row, float s, int half,
-                                                 uint32_t (&outr)[16]) {
+__device__ __forceinline__ void dequant_half_row(const uint8_t* row, int sw7, int s, int half,
+                                                 float scale, uint32_t (&outr)[16]) {
+  auto piece = [&](int j) {
+    return *reinterpret_cast<const uint4*>(row + ((j ^ sw7) << 4));
+  };
   uint4 out[4];
   if constexpr (FMT == 4) {
-    const uint4 q = *reinterpret_cast<const uint4*>(raw_row + 16 * half);
+    const uint4 q = piece(2 * s + half);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    const __half2 s2 = __float2half2_rn(s);
+    const __half2 s2 = __float2half2_rn(scale);
     const __half2 bias = __float2half2_rn(1032.f);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {  // word j = K values 8j .. 8j+7 of this half
@@ -342,14 +379,14 @@ __device__ __forceinline__ void dequant_half_row(const uint8_t* raw_row, float s
       out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
     }
   } else if constexpr (FMT == 8) {
-    const uint4 q0 = *reinterpret_cast<const uint4*>(raw_row + 32 * half);
-    const uint4 q1 = *reinterpret_cast<const uint4*>(raw_row + 32 * half + 16);
+    const uint4 q0 = piece(4 * s + 2 * half);
+    const uint4 q1 = piece(4 * s + 2 * half + 1);
     const uint32_t qq[8] = {q0.x ^ 0x80808080u, q0.y ^ 0x80808080u, q0.z ^ 0x80808080u,
                             q0.w ^ 0x80808080u, q1.x ^ 0x80808080u, q1.y ^ 0x80808080u,
                             q1.z ^ 0x80808080u, q1.w ^ 0x80808080u};  // u = q + 128 per byte
     // 0x4B000000 | u is the fp32 value 2^23 + u; fma((2^23 + u), s, -(2^23 + 128) s) = q s,
     // exact (the constant needs 24 significant bits at most), then one rounding to fp16.
-    const float c = -8388736.f * s;
+    const float c = -8388736.f * scale;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {  // piece j = bytes 8j .. 8j+7 = words 2j, 2j+1
       uint32_t pr[4];
@@ -359,7 +396,7 @@ __device__ __forceinline__ void dequant_half_row(const uint8_t* raw_row, float s
         const int b0 = 2 * (i & 1);
         const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | b0));
         const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | (b0 + 1)));
-        __half2 h = __floats2half2_rn(fmaf(f0, s, c), fmaf(f1, s, c));
+        __half2 h = __floats2half2_rn(fmaf(f0, scale, c), fmaf(f1, scale, c));
         pr[i] = *reinterpret_cast<uint32_t*>(&h);
       }
       out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
@@ -367,7 +404,7 @@ __device__ __forceinline__ void dequant_half_row(const uint8_t* raw_row, float s
   } else {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint4 v = *reinterpret_cast<const uint4*>(raw_row + 64 * half + 16 * j);
+      const uint4 v = piece(4 * half + j);
       const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
       uint32_t pr[4];
 #pragma unroll
@@ -406,8 +443,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* full_x = empty_w + C::NW;        // [NX]
   uint64_t* empty_x = full_x + C::NX;        // [NX]
   uint64_t* full_a = empty_x + C::NX;        // [NA]
-  uint64_t* empty_a = full_a + C::NA;        // [NA]
-  uint64_t* acc_full = empty_a + C::NA;      // [2]
+  uint64_t* acc_full = full_a + C::NA;       // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
   uint64_t* scale_full = acc_empty + 2;      // [2] one per unit parity
   uint64_t* scale_empty = scale_full + 2;    // [2]
@@ -421,29 +457,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int G = K / kGroup;
   const int n_tiles = N / kTcM;
   const int n_chunks = K / kTcBK;
+  const int n_wstages = (n_chunks + C::SUB - 1) / C::SUB;  // weight stages a unit
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NW; ++s) {
       mbar_init(&full_w[s], 1);
       mbar_init(&empty_w[s], kDqWarps);  // dequant warps
     }
+    // a chunk's activation stage and A stage are released together by one commit of each
+    // MMA issuer (the rings have the same depth and advance in step)
     for (int s = 0; s < C::NX; ++s) {
       mbar_init(&full_x[s], 1);
-      mbar_init(&empty_x[s], NM);        // one MMA commit per issuer
+      mbar_init(&empty_x[s], kIssuers);
     }
-    for (int s = 0; s < C::NA; ++s) {
-      mbar_init(&full_a[s], kDqWarps);  // dequant warps
-      mbar_init(&empty_a[s], NM);       // one MMA commit per issuer
-    }
+    for (int s = 0; s < C::NA; ++s) mbar_init(&full_a[s], kDqWarps / 2);  // one group
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], NM);      // one MMA commit per issuer
+      mbar_init(&acc_full[b], kIssuers);  // one MMA commit per issuer
       mbar_init(&acc_empty[b], 4);      // 4 epilogue warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&scale_full[b], 1);
       mbar_init(&scale_empty[b], kDqWarps);
     }
-    mbar_init(drain, NM);
+    mbar_init(drain, kIssuers);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -482,14 +518,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producers
+    // Lane 0 streams the weights (and each unit's scales), gated only by the dequantisers
+    // releasing weight stages, so it runs up to NW stages ahead; warp 15 streams the
+    // activation tiles, gated by the tensor core releasing them. Coupling both to one loop
+    // (or to two lanes of one warp, which then take turns) holds one back by the other.
     if (lane == 0) {
       int it = 0, ui = 0;
       for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++ui) {
         const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
-        const int bx = box_index(t.nrows);
         const int src = t.shared ? 1 : 0;
-        const int box_rows = maps.box_rows[src][bx];
         const int wrow = t.e * N + t.ntile * kTcM;
         TCT(0, ui, 0);
         if constexpr (FMT != 16) {
@@ -508,36 +546,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      (uint32_t)SL.sb, &scale_full[sbuf]);
           }
         }
-        for (int c = 0; c < n_chunks; ++c, ++it) {
+        bool ok = true;
+        for (int cw = 0; cw < n_wstages; ++cw, ++it) {
           const int sw = it % C::NW, uw = it / C::NW;
-          const int sx = it % C::NX, ux = it / C::NX;
-          if ((uw > 0 && !mbar_wait(&empty_w[sw], (uw - 1) & 1)) ||
-              (ux > 0 && !mbar_wait(&empty_x[sx], (ux - 1) & 1))) {
-            fail();
+          if (uw > 0 && !mbar_wait(&empty_w[sw], (uw - 1) & 1)) {
+            ok = false;
             break;
           }
+          // a partial last stage reads past the row end: the TMA fills zeros there and
+          // still counts the whole box
           mbar_arrive_expect_tx(&full_w[sw], (uint32_t)C::WB);
 #pragma unroll
           for (int mi = 0; mi < NM; ++mi)
             tma_load_2d(smem + C::R_OFF + sw * C::WB + mi * C::RAW, &maps.w[src][mi],
-                        c * C::RAW_ROW, wrow, &full_w[sw]);
-          mbar_arrive_expect_tx(&full_x[sx], (uint32_t)(box_rows * kTcBK * 2));
-          tma_load_2d(smem + C::X_OFF + sx * C::XB, &maps.act[src][bx], c * kTcBK, t.row0,
-                      &full_x[sx]);
+                        cw * C::RAW_ROW, wrow, &full_w[sw]);
+        }
+        if (!ok) {
+          fail();
+          break;
         }
         TCT(0, ui, 1);
       }
-      // every issued copy lands before the CTA may exit (consumed ones already have)
+      // every issued stage lands before the CTA may exit (consumed ones already have)
       for (int j = (it > C::NW ? it - C::NW : 0); j < it; ++j)
         mbar_wait(&full_w[j % C::NW], (j / C::NW) & 1);
-      for (int j = (it > C::NX ? it - C::NX : 0); j < it; ++j)
-        mbar_wait(&full_x[j % C::NX], (j / C::NX) & 1);
     }
+    __syncwarp();
   } else if (warp == 1 || warp == 14) {
     // ------------------------------------------------------------ MMA issuers
-    const int mi = (warp == 1) ? 0 : 1;  // matrix this thread issues
-    if (lane == 0 && mi < NM) {
-      int it = 0, ia = 0, tile = 0;
+    // Two threads issue (the issue cost of a tcgen05.mma is mostly per-thread latency):
+    // gate/up: issuer i takes matrix i, all K steps; down: issuer i takes the K steps
+    // 2i, 2i+1 of every chunk into its own accumulator (the epilogue adds the two).
+    const int iss = (warp == 1) ? 0 : 1;
+    if (lane == 0) {
+      const int mi = GATE_UP ? iss : 0;
+      const int k0 = GATE_UP ? 0 : 2 * iss, k1 = GATE_UP ? kTcBK / 16 : 2 * iss + 2;
+      int it = 0, tile = 0;
       for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
         const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
         const int n_mma = (t.nrows + 15) & ~15;
@@ -549,28 +593,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
         TCT(1, tile, 0);
-        const uint32_t d0 = tmem + b * 128;  // gate (or down) accumulator; up at +64
+        const uint32_t dacc = tmem + b * 128 + iss * kTcNMax;  // this issuer's accumulator
         bool ok = true;
-        for (int c = 0; c < n_chunks; ++c, ++it, ++ia) {
-          const int sx = it % C::NX, a = ia % C::NA;
-          const bool okx = mbar_wait(&full_x[sx], (it / C::NX) & 1);
+        for (int c = 0; c < n_chunks; ++c, ++it) {
+          const int s = it % C::NX;
+          const bool okx = mbar_wait(&full_x[s], (it / C::NX) & 1);
           TCC(it, 0);
-          const bool oka = okx && mbar_wait(&full_a[a], (ia / C::NA) & 1);
+          const bool oka = okx && mbar_wait(&full_a[s], (it / C::NA) & 1);
           TCC(it, 1);
           if (!oka) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t xs = smem_u32(smem + C::X_OFF + sx * C::XB);
+          // One descriptor and one TMEM address per chunk; the K steps advance them by
+          // constants (32 bytes of B = 2 in the descriptor's address field, 8 columns of A).
+          const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::X_OFF + s * C::XB));
+          const uint32_t at = tmem + C::A_COL0 + s * C::A_COLS + mi * (kTcBK / 2);
+          umma_f16_ts(dacc, at + k0 * 8, bdesc + (uint64_t)(2 * k0), idesc, c > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < kTcBK / 16; ++kk) {
-            const uint64_t bdesc = umma_desc_sw128(xs + kk * 32);
-            const uint32_t at = tmem + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2) + kk * 8;
-            umma_f16_ts(d0 + mi * kTcNMax, at, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&empty_x[sx]);
-          umma_commit(&empty_a[a]);
+          for (int kk = 1; kk < kTcBK / 16; ++kk)
+            if (k0 + kk < k1)
+              umma_f16_ts_acc(dacc, at + (k0 + kk) * 8, bdesc + (uint64_t)(2 * (k0 + kk)), idesc);
+          umma_commit(&empty_x[s]);  // releases the activation stage and the A stage
           TCC(it, 2);
         }
         if (!ok) {
@@ -586,9 +631,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < 2 + kDqWarps) {
     // ------------------------------------------------------------ dequantisers
-    // TMEM lanes a warp may write are 32 * (warp % 4) .. +31: rows follow the warp
+    // Two groups of four warps take alternate chunks (group g: chunks c with c % 2 == g), so
+    // two chunks are converted at a time; within a group, warp w covers the weight rows of
+    // TMEM lanes 32 * (w % 4) .. +31 (the lanes a warp may write), both K halves.
     const int r = 32 * (warp & 3) + lane;            // weight row in the tile
-    const int half = (warp - 2) >> 2;                // which 32 K values of the chunk
+    const int group = (warp - 2) >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     int it = 0, ia = 0, ui = 0;
     for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++ui) {
@@ -597,36 +644,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (threadIdx.x == 64) TCT(2, ui, 0);
       if constexpr (FMT != 16) ok = mbar_wait(&scale_full[sbuf], (ui >> 1) & 1);
       const uint16_t* sblk = reinterpret_cast<const uint16_t*>(smem + C::S_OFF + sbuf * NM * SL.sb);
-      for (int c = 0; c < n_chunks && ok; ++c, ++it, ++ia) {
-        const int sw = it % C::NW, a = ia % C::NA;
-        float sc[NM];
-#pragma unroll
-        for (int mi = 0; mi < NM; ++mi)
-          sc[mi] = (FMT == 16) ? 1.f
-                               : bf16_to_f32(sblk[mi * (SL.sb / 2) + r * G + (c * kTcBK) / kGroup]);
-        const bool okw = mbar_wait(&full_w[sw], (it / C::NW) & 1);
-        if (threadIdx.x == 64) TCC(it, 3);
-        const bool oka = okw && (ia < C::NA || mbar_wait(&empty_a[a], ((ia / C::NA) - 1) & 1));
-        if (threadIdx.x == 64) TCC(it, 4);
-        if (!oka) {
+      for (int cw = 0; cw < n_wstages && ok; ++cw, ++it) {
+        const int sw = it % C::NW;
+        // every warp waits for every stage before releasing it (keeps the release phases
+        // of the stage in order, also for a group with no chunk in it)
+        if (!mbar_wait(&full_w[sw], (it / C::NW) & 1)) {
           ok = false;
           break;
         }
+        const int c_end = min(n_chunks, (cw + 1) * C::SUB);
+        for (int c = cw * C::SUB; c < c_end; ++c, ++ia) {
+          if ((c & 1) != group) continue;
+          const int a = ia % C::NA;
+          float sc[NM];
 #pragma unroll
-        for (int mi = 0; mi < NM; ++mi) {
-          const uint8_t* raw_row = smem + C::R_OFF + sw * C::WB + mi * C::RAW + r * C::RAW_ROW;
-          uint32_t regs[16];
-          dequant_half_row<FMT>(raw_row, sc[mi], half, regs);
-          tmem_st16(lane_base + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2) + 16 * half, regs);
+          for (int mi = 0; mi < NM; ++mi)
+            sc[mi] = (FMT == 16) ? 1.f
+                                 : bf16_to_f32(sblk[mi * (SL.sb / 2) + r * G + (c * kTcBK) / kGroup]);
+          if (threadIdx.x == 64) TCC(ia, 3);
+          if (ia >= C::NA && !mbar_wait(&empty_x[a], ((ia / C::NA) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          if (threadIdx.x == 64) TCC(ia, 4);
+#pragma unroll
+          for (int mi = 0; mi < NM; ++mi) {
+            const uint8_t* raw_row = smem + C::R_OFF + sw * C::WB + mi * C::RAW + r * C::RAW_ROW;
+            uint32_t regs[32];
+            uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[0]);
+            uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[16]);
+            dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 0, sc[mi], lo);
+            dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 1, sc[mi], hi);
+            tmem_st32(lane_base + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2), regs);
+          }
+          tmem_st_wait();
+          tc_fence_before();  // the stores are complete before the arrive below
+          __syncwarp();
+          if (threadIdx.x == 64) TCC(ia, 5);
+          if (lane == 0) mbar_arrive(&full_a[a]);
         }
-        tmem_st_wait();
-        tc_fence_before();  // the stores are complete before the arrive below
         __syncwarp();
-        if (threadIdx.x == 64) TCC(it, 5);
-        if (lane == 0) {
-          mbar_arrive(&full_a[a]);
-          mbar_arrive(&empty_w[sw]);
-        }
+        if (lane == 0) mbar_arrive(&empty_w[sw]);  // the stage is read
       }
       if (!ok) {
         fail();
@@ -638,6 +696,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (threadIdx.x == 64) TCT(2, ui, 1);
     }
+  } else if (warp == 15) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      int it = 0;
+      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+        const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
+        const int bx = box_index(t.nrows);
+        const int src = t.shared ? 1 : 0;
+        const int box_rows = maps.box_rows[src][bx];
+        bool ok = true;
+        for (int c = 0; c < n_chunks; ++c, ++it) {
+          const int sx = it % C::NX, ux = it / C::NX;
+          if (ux > 0 && !mbar_wait(&empty_x[sx], (ux - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_x[sx], (uint32_t)(box_rows * kTcBK * 2));
+          tma_load_2d(smem + C::X_OFF + sx * C::XB, &maps.act[src][bx], c * kTcBK, t.row0,
+                      &full_x[sx]);
+        }
+        if (!ok) {
+          fail();
+          break;
+        }
+      }
+      for (int j = (it > C::NX ? it - C::NX : 0); j < it; ++j)
+        mbar_wait(&full_x[j % C::NX], (j / C::NX) & 1);
+    }
+    __syncwarp();
   } else if (warp < 14) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31 (warps 10..13)
@@ -671,6 +758,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           }
         } else {
+          float g2[16];
+          tmem_ld16(lane_addr + kTcNMax + m0, g2);  // the second issuer's K steps
+#pragma unroll
+          for (int j = 0; j < 16; ++j) g[j] += g2[j];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (m0 + j < t.nrows) {
@@ -762,7 +853,7 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
       const int which = GATE_UP ? mi : 2;
       if (!make_map(&maps.w[b][mi], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, banks[b]->w[which],
                     wbytes_per_row, (uint64_t)nexp[b] * N, box_w, kTcM,
-                    CU_TENSOR_MAP_SWIZZLE_NONE))
+                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     }
   }

@@ -73,8 +73,8 @@ typedef enum {
 typedef enum { MOE_W_BF16 = 16, MOE_W_INT8 = 8, MOE_W_INT4 = 4 } moe_wfmt;
 
 /* Which kernels run. AUTO picks the single-kernel layer (FUSED) for 1-token calls with
- * int4 banks when the device fits it, the split-K GEMV kernels for other calls of 1..32
- * rows, and the tensor-core (tcgen05) grouped GEMMs for larger token counts. FUSED asks for
+ * int4 banks when the device fits it, the split-K GEMV kernels for other calls of 1..15
+ * rows, and the tensor-core (tcgen05) grouped GEMMs from 16 rows up. FUSED asks for
  * the single-kernel layer and returns MOE_ERR_UNSUPPORTED from moe_layer_forward when the
  * call does not fit it; the stage entry points (moe_route ... moe_combine) treat FUSED like
  * GEMV. */
