@@ -65,65 +65,115 @@ __global__ void __launch_bounds__(256) router_small_kernel(
 }
 
 // ------------------------------------------------------------------ logits, many tokens
-// Classic shared-memory tiled SIMT product: 64 tokens x 64 experts per CTA, K step 32,
-// 256 threads with a 4x4 register tile each.
-constexpr int kRT = 64, kRE = 64, kRK = 32;
+// Tensor-core product (mma.sync m16n8k16, bf16 inputs, fp32 accumulation; the products of
+// two bf16 values are exact in fp32): 64 tokens x 64 experts per CTA, 4 warps of 32 x 32,
+// K in tiles of 64 staged by 16-byte cp.async copies (double buffered, rows padded to 72
+// elements so the 8 rows an ldmatrix reads fall in distinct banks). Each logit is summed
+// in one fixed order, so the result is reproducible.
+constexpr int kRT = 64, kRE = 64, kRK = 64, kRPad = 72;
 
-__global__ void __launch_bounds__(256) router_tiled_kernel(
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+}
+
+__global__ void __launch_bounds__(128) router_mma_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ wr,
     const float* __restrict__ bias, float* __restrict__ logits, int T, int d, int E) {
-  __shared__ float xs[kRK][kRT + 4];
-  __shared__ float ws[kRK][kRE + 4];
+  __shared__ __align__(16) uint16_t xs[2][kRT][kRPad];
+  __shared__ __align__(16) uint16_t ws[2][kRE][kRPad];
   const int t0 = blockIdx.y * kRT, e0 = blockIdx.x * kRE;
-  const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;  // 16 x 16 threads, 4 x 4 each
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < d; k0 += kRK) {
-    // load 64 x 32 of X and of Wr: 2048 elements each, 8 per thread
-    for (int i = tid; i < kRT * kRK / 8; i += 256) {
-      const int row = i / (kRK / 8), c8 = i % (kRK / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t0 + row < T) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + row) * d + k0) + c8);
-      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wt = (warp >> 1) * 32, we = (warp & 1) * 32;  // this warp's 32 x 32 block
+
+  // tile k0 -> stage s: 64 rows x 8 pieces of 16 bytes for X and for Wr (1024 copies, 8 a
+  // thread); rows past T or E read nothing and fill zeros
+  auto load = [&](int s, int k0) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        xs[c8 * 8 + 2 * q][row] = __uint_as_float(vv[q] << 16);
-        xs[c8 * 8 + 2 * q + 1][row] = __uint_as_float(vv[q] & 0xffff0000u);
-      }
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (e0 + row < E) w = __ldg(reinterpret_cast<const uint4*>(wr + (size_t)(e0 + row) * d + k0) + c8);
-      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        ws[c8 * 8 + 2 * q][row] = __uint_as_float(wv[q] << 16);
-        ws[c8 * 8 + 2 * q + 1][row] = __uint_as_float(wv[q] & 0xffff0000u);
+    for (int i = 0; i < 8; ++i) {
+      const int c = tid + 128 * i;  // 0 .. 1023
+      const int which = c >> 9, row = (c >> 3) & 63, piece = c & 7;
+      if (which == 0) {
+        const int t = t0 + row;
+        const uint16_t* src = x + (size_t)min(t, T - 1) * d + k0 + 8 * piece;
+        cp_async16(&xs[s][row][8 * piece], src, t < T ? 16 : 0);
+      } else {
+        const int e = e0 + row;
+        const uint16_t* src = wr + (size_t)min(e, E - 1) * d + k0 + 8 * piece;
+        cp_async16(&ws[s][row][8 * piece], src, e < E ? 16 : 0);
       }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  float acc[2][4][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][j][q] = 0.f;
+
+  const int n_k = d / kRK;
+  load(0, 0);
+  for (int kt = 0; kt < n_k; ++kt) {
+    const int s = kt & 1;
+    if (kt + 1 < n_k) {
+      load(s ^ 1, (kt + 1) * kRK);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kRK; ++kk) {
-      float a[4], b[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
+    for (int kk = 0; kk < kRK; kk += 16) {
+      // A (tokens x K, row-major): two 16 x 16 fragments; B (experts x K = the K-major "col"
+      // operand): four 8-expert x 16 fragments, two per ldmatrix.x4
+      uint32_t a[2][4], b[2][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = ws[kk][tx * 4 + j];
+      for (int i = 0; i < 2; ++i)
+        ldmatrix_x4(a[i], &xs[s][wt + 16 * i + (lane & 15)][kk + 8 * (lane >> 4)]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 2; ++j)
+        ldmatrix_x4(b[j], &ws[s][we + 16 * j + (lane & 7) + 8 * (lane >> 4)][kk + 8 * ((lane >> 3) & 1)]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t b0 = b[j >> 1][2 * (j & 1)], b1 = b[j >> 1][2 * (j & 1) + 1];
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+              "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+              : "+f"(acc[i][j][0]), "+f"(acc[i][j][1]), "+f"(acc[i][j][2]), "+f"(acc[i][j][3])
+              : "r"(a[i][0]), "r"(a[i][1]), "r"(a[i][2]), "r"(a[i][3]), "r"(b0), "r"(b1));
+        }
     }
     __syncthreads();
   }
+  // C fragment: rows grp and grp + 8 of the 16-token block, columns 2q, 2q + 1 of the 8
+  const int grp = lane >> 2, q = lane & 3;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= T) continue;
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.f);
-    }
-  }
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = t0 + wt + 16 * i + grp + 8 * h;
+        if (t >= T) continue;
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int e = e0 + we + 8 * j + 2 * q + c2;
+          if (e < E) logits[(size_t)t * E + e] = acc[i][j][2 * h + c2] + (bias ? bias[e] : 0.f);
+        }
+      }
 }
 
 cudaError_t launch_router(const Plan& p, cudaStream_t st) {
@@ -134,8 +184,8 @@ cudaError_t launch_router(const Plan& p, cudaStream_t st) {
                                                 p.d, p.E);
   } else {
     dim3 grid((p.E + kRE - 1) / kRE, (p.T + kRT - 1) / kRT);
-    router_tiled_kernel<<<grid, 256, 0, st>>>(p.x, p.router_w, p.router_bias, p.logits, p.T,
-                                              p.d, p.E);
+    router_mma_kernel<<<grid, 128, 0, st>>>(p.x, p.router_w, p.router_bias, p.logits, p.T, p.d,
+                                            p.E);
   }
   return cudaGetLastError();
 }
