@@ -84,6 +84,11 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Arrives at named barrier `id` (of `threads` threads) without waiting; whole warps only.
+__device__ __forceinline__ void named_bar_arrive(int id, int threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 #ifdef MOE_TRACE
 // Kernel timeline (trace builds only): per kernel id, earliest entry, earliest and latest
 // return from the dependency wait, latest exit, in globaltimer nanoseconds.

@@ -12,9 +12,9 @@
 // One persistent CTA per SM, warp roles:
 //   warp 0      TMA producer of the raw weight stages [128 rows x 128 bytes] (int4/int8/
 //               bf16, 128-byte swizzle) and each unit's group scales
-//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16, fp32
-//               accumulate; for gate/up warp 14 issues the up-projection MMAs in parallel
-//               (separate accumulator), which halves the instructions one thread issues
+//   warp 1      TMEM owner and MMA issuer (the whole warp, one elected lane issuing):
+//               tcgen05.mma kind::f16, fp32 accumulate; warp 14 issues in parallel into a
+//               separate accumulator (gate/up: the up projection; down: half the K steps)
 //   warps 2-9   dequantisers, two groups of four taking alternate chunks: W = fp16(q * s)
 //               written straight from registers into TMEM (tcgen05.st), where the MMA
 //               reads its A operand;
@@ -25,8 +25,9 @@
 // Operands are fp16 (kind::f16, fp32 accumulate): the activations (bf16 inputs) convert to
 // fp16 exactly in fp16's range, and q * s rounds once with an 11-bit significand, eight
 // times finer than bf16. Activations and h outside fp16's range set a device status flag.
-// Rings: weights (TMA -> dequant), activations (TMA -> MMA), A (dequant -> MMA, in TMEM),
-// accumulator (MMA -> epilogue, double buffered in TMEM). TMEM columns: accumulators
+// Rings: weights (TMA -> dequant), activations (TMA -> MMA), A (dequant -> MMA, in TMEM;
+// announced on a named barrier per stage), accumulator (MMA -> epilogue, double buffered in
+// TMEM). TMEM columns: accumulators
 // [0, 256) (buffer b: gate at 128 b, up at 128 b + 64), A stages [256, 512). Every wait is bounded; a timeout sets the
 // status word and every role drains and exits (TMEM is freed by its owner).
 //
@@ -65,7 +66,9 @@ extern "C" __attribute__((visibility("default"))) int moe_tct_read(void* dst) {
 
 constexpr int kTcThreads = 512;  // 16 warps
 constexpr int kDqWarps = 8;       // dequantisers (two threads per weight row)
-constexpr int kIssuers = 2;       // MMA issuing threads (warps 1 and 14)
+constexpr int kIssuers = 2;       // MMA issuing warps (1 and 14)
+// threads of one chunk's ready barrier: a dequantiser group of four warps and the issuers
+constexpr int kReadyThreads = 32 * (kDqWarps / 2 + kIssuers);
 constexpr int kTcBK = 64;      // K per chunk (one 128-byte swizzle span of bf16)
 constexpr int kTcM = 128;      // weight rows per tile
 constexpr int kTcNMax = 64;    // token rows per tile
@@ -97,6 +100,7 @@ template <int FMT, bool GATE_UP> struct TcCfg {
   static constexpr int NA = NX;                      // A stages in TMEM
   static constexpr int A_COL0 = 256;
   static_assert(A_COL0 + NA * A_COLS <= 512, "TMEM budget");
+  static_assert(NX <= 15, "one named barrier per stage (ids 1..15)");
   // layout (1024-byte aligned pieces first)
   static constexpr int X_OFF = 0;
   static constexpr int R_OFF = X_OFF + NX * XB;
@@ -154,48 +158,30 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
+// Warp-level forms: the whole (converged) warp executes them and one elected lane issues.
+// Issuing from a converged warp costs a fraction of issuing from a lone lane of a diverged
+// warp (about 17 against 46 cycles per M = 128, N = 16 MMA). elect.sync picks the lowest
+// active lane, the same thread every time, so the MMAs and their commits stay in one
+// thread's issue order.
+__device__ __forceinline__ void umma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// A operand from TMEM (row = lane, K packed two fp16 per 32-bit column), B from shared memory.
-__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-// The same, accumulating into D unconditionally (no per-instruction predicate set-up).
-__device__ __forceinline__ void umma_f16_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                                uint32_t idesc) {
+__device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 1, 1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc)
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
       : "memory");
 }
 
-// 16 consecutive 32-bit columns of this thread's TMEM lane <- registers.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-      "%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-
-// 32 consecutive 32-bit columns of this thread's TMEM lane <- registers (one instruction:
-// tcgen05 instructions cost each issuing thread about a hundred cycles or more).
+// 32 consecutive 32-bit columns of this thread's TMEM lane <- registers (one wide
+// instruction: every tcgen05 instruction has a sizeable fixed issue cost).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
@@ -210,13 +196,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
 }
 
 // 16 consecutive fp32 columns of this thread's TMEM lane.
@@ -283,6 +262,19 @@ __device__ __forceinline__ int box_index(int nrows) {
   return nrows <= 16 ? 0 : (nrows <= 32 ? 1 : (nrows <= 64 ? 2 : 3));
 }
 
+// K order of the fp16 operands the tensor core reads. For int4 weights the dequantisers
+// produce K pairs interleaved by four inside each aligned group of 8 (operand position 2i holds
+// K 8m+i, position 2i+1 holds K 8m+i+4), so the activation rows multiplied with such a bank
+// (x rows for gate/up, h rows for down) are stored in that order too; other formats keep K in
+// order. A shared permutation of K leaves the contraction unchanged.
+__host__ __device__ __forceinline__ bool interleaved_k(int fmt) { return fmt == 4; }
+
+// Operand position of K index n (the position within its aligned group of 8 changes only).
+__device__ __forceinline__ int k_position(int n, bool interleave) {
+  const int i = n & 7;
+  return interleave ? ((n & ~7) | ((i & 3) << 1) | (i >> 2)) : n;
+}
+
 // Gathers the activation rows in fp16 (xg[r] = x[perm[r] / k] for the T*k grouped rows, then
 // xg[T*k + t] = x[t] for the shared expert) and, in CTA 0, builds the unit schedule.
 __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_t* xg) {
@@ -326,14 +318,20 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
          i += (size_t)gridDim.x * blockDim.x) {
       const int r = (int)(i / chunks), c = (int)(i % chunks);
       const int t = (r < n) ? p.perm[r] / p.k : r - n;
+      const bool il = interleaved_k((r < n) ? p.routed.fmt : p.shared.fmt);
       const uint4 v = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d)[c];
       const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+      float e[8];  // K values 8c .. 8c+7
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        e[2 * q] = __uint_as_float(vv[q] << 16);
+        e[2 * q + 1] = __uint_as_float(vv[q] & 0xffff0000u);
+        range_ok &= (fabsf(e[2 * q]) <= 65504.f) && (fabsf(e[2 * q + 1]) <= 65504.f);
+      }
       uint32_t o[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float a = __uint_as_float(vv[q] << 16), b = __uint_as_float(vv[q] & 0xffff0000u);
-        range_ok &= (fabsf(a) <= 65504.f) && (fabsf(b) <= 65504.f);
-        __half2 h = __floats2half2_rn(a, b);
+        __half2 h = il ? __floats2half2_rn(e[q], e[q + 4]) : __floats2half2_rn(e[2 * q], e[2 * q + 1]);
         o[q] = *reinterpret_cast<uint32_t*>(&h);
       }
       reinterpret_cast<uint4*>(xg + (size_t)r * p.d)[c] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -346,82 +344,72 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
 // ------------------------------------------------------------------ dequantisation
 
 // Half `half` (K values 32*half .. 32*half+31) of chunk `s` (K values 64*s .. 64*s+63 of the
-// stage) of one weight row -> 32 fp16 = W * s in K order, two per register. The row is one
-// 128-byte line of a stage written by the TMA with 128-byte swizzling: its 16-byte piece j
-// sits at piece j ^ sw7 (sw7 = the row index mod 8).
+// stage) of one weight row -> 32 fp16 = W * s, two per register. The row is one 128-byte
+// line of a stage written by the TMA with 128-byte swizzling: its 16-byte piece j sits at
+// piece j ^ sw7 (sw7 = the row index mod 8).
+//
+// int4 registers hold K pairs interleaved by four inside each 8-value word: register i of
+// word j = (K 8j+i, K 8j+i+4), i = 0..3 (interleaved_k; the activation rows carry the
+// same order, so the contraction is unchanged). That order needs only masks: the integer
+// pipe, which issues a warp instruction every other cycle, does 5 instructions per 8
+// weights instead of 9 for the K-ordered pairs. int8 and bf16 registers hold K in order.
+//
+// Every conversion is exact up to one final rounding of q * s to fp16 (for scales in fp16's
+// normal range): a nibble or byte placed in the mantissa of 1024.0 gives 1024 + u exactly,
+// the offset is taken off exactly, and one fp16 multiply rounds q * s.
 template <int FMT>
 __device__ __forceinline__ void dequant_half_row(const uint8_t* row, int sw7, int s, int half,
                                                  float scale, uint32_t (&outr)[16]) {
   auto piece = [&](int j) {
     return *reinterpret_cast<const uint4*>(row + ((j ^ sw7) << 4));
   };
-  uint4 out[4];
+  auto h2 = [](uint32_t u) { return *reinterpret_cast<__half2*>(&u); };
+  auto u32 = [](__half2 h) { return *reinterpret_cast<uint32_t*>(&h); };
   if constexpr (FMT == 4) {
     const uint4 q = piece(2 * s + half);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
     const __half2 s2 = __float2half2_rn(scale);
-    const __half2 bias = __float2half2_rn(1032.f);
+    const __half2 off = __float2half2_rn(1032.f), sixteenth = __float2half2_rn(0.0625f),
+                  off16 = __float2half2_rn(-72.f);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {  // word j = K values 8j .. 8j+7 of this half
-      const uint32_t lo = w[j], hi = w[j] >> 4;
-      uint32_t pr[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        // byte i of lo holds nibble 2i in its low half, byte i of hi holds nibble 2i+1;
-        // keep those two nibbles, flip their sign bit and place them in the mantissa of
-        // 1024.0: fp16 values 1024 + (n ^ 8) = q + 1032, exact
-        uint32_t t = __byte_perm(lo, hi, i | ((4 + i) << 8));
-        t = (t & 0x000F000Fu) ^ 0x64086408u;
-        __half2 v = *reinterpret_cast<__half2*>(&t);
-        v = __hmul2(__hsub2(v, bias), s2);  // q exact, then one rounding of q * s
-        pr[i] = *reinterpret_cast<uint32_t*>(&v);
-      }
-      out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+    for (int j = 0; j < 4; ++j) {  // word j = K values 8j .. 8j+7 of this half, nibble i = K 8j+i
+      const uint32_t lo = w[j], hi = w[j] >> 8;
+      // (n & 15) ^ 8 = q + 8 (offset binary) in the low mantissa bits of 1024.0, two at a time:
+      // nibbles 0/4 (and 2/6 of hi) as 1024 + (q + 8), nibbles 1/5 (3/7) as 1024 + 16 (q + 8)
+      const uint32_t a = (lo & 0x000F000Fu) ^ 0x64086408u;
+      const uint32_t b = (lo & 0x00F000F0u) ^ 0x64806480u;
+      const uint32_t c = (hi & 0x000F000Fu) ^ 0x64086408u;
+      const uint32_t d = (hi & 0x00F000F0u) ^ 0x64806480u;
+      outr[4 * j + 0] = u32(__hmul2(__hsub2(h2(a), off), s2));             // K 8j+0, 8j+4
+      outr[4 * j + 1] = u32(__hmul2(__hfma2(h2(b), sixteenth, off16), s2));  // 8j+1, 8j+5
+      outr[4 * j + 2] = u32(__hmul2(__hsub2(h2(c), off), s2));             // 8j+2, 8j+6
+      outr[4 * j + 3] = u32(__hmul2(__hfma2(h2(d), sixteenth, off16), s2));  // 8j+3, 8j+7
     }
   } else if constexpr (FMT == 8) {
     const uint4 q0 = piece(4 * s + 2 * half);
     const uint4 q1 = piece(4 * s + 2 * half + 1);
-    const uint32_t qq[8] = {q0.x ^ 0x80808080u, q0.y ^ 0x80808080u, q0.z ^ 0x80808080u,
-                            q0.w ^ 0x80808080u, q1.x ^ 0x80808080u, q1.y ^ 0x80808080u,
-                            q1.z ^ 0x80808080u, q1.w ^ 0x80808080u};  // u = q + 128 per byte
-    // 0x4B000000 | u is the fp32 value 2^23 + u; fma((2^23 + u), s, -(2^23 + 128) s) = q s,
-    // exact (the constant needs 24 significant bits at most), then one rounding to fp16.
-    const float c = -8388736.f * scale;
+    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const __half2 s2 = __float2half2_rn(scale);
+    const __half2 off = __float2half2_rn(1152.f);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {  // piece j = bytes 8j .. 8j+7 = words 2j, 2j+1
-      uint32_t pr[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t w = qq[2 * j + (i >> 1)];
-        const int b0 = 2 * (i & 1);
-        const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | b0));
-        const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | (b0 + 1)));
-        __half2 h = __floats2half2_rn(fmaf(f0, scale, c), fmaf(f1, scale, c));
-        pr[i] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+    for (int j = 0; j < 8; ++j) {  // word j = K values 4j .. 4j+3
+      const uint32_t u = w[j] ^ 0x80808080u;  // byte = q + 128
+      // bytes 0, 1 (2, 3) with 0x64 above each: fp16 pair 1024 + q + 128, exact
+      const uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);
+      const uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);
+      outr[2 * j] = u32(__hmul2(__hsub2(h2(a), off), s2));
+      outr[2 * j + 1] = u32(__hmul2(__hsub2(h2(b), off), s2));
     }
   } else {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint4 v = piece(4 * half + j);
       const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-      uint32_t pr[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __half2 h = __floats2half2_rn(__uint_as_float(vv[i] << 16),
-                                      __uint_as_float(vv[i] & 0xffff0000u));
-        pr[i] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      out[j] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+      for (int i = 0; i < 4; ++i)
+        outr[4 * j + i] = u32(__floats2half2_rn(__uint_as_float(vv[i] << 16),
+                                                __uint_as_float(vv[i] & 0xffff0000u)));
     }
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    outr[4 * j] = out[j].x;
-    outr[4 * j + 1] = out[j].y;
-    outr[4 * j + 2] = out[j].z;
-    outr[4 * j + 3] = out[j].w;
   }
 }
 
@@ -442,8 +430,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* empty_w = full_w + C::NW;        // [NW]
   uint64_t* full_x = empty_w + C::NW;        // [NX]
   uint64_t* empty_x = full_x + C::NX;        // [NX]
-  uint64_t* full_a = empty_x + C::NX;        // [NA]
-  uint64_t* acc_full = full_a + C::NA;       // [2]
+  uint64_t* acc_full = empty_x + C::NX;      // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
   uint64_t* scale_full = acc_empty + 2;      // [2] one per unit parity
   uint64_t* scale_empty = scale_full + 2;    // [2]
@@ -465,12 +452,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&empty_w[s], kDqWarps);  // dequant warps
     }
     // a chunk's activation stage and A stage are released together by one commit of each
-    // MMA issuer (the rings have the same depth and advance in step)
+    // MMA issuer (the rings have the same depth and advance in step); a chunk is announced
+    // ready to the issuers on named barrier 1 + stage (kReadyThreads threads)
     for (int s = 0; s < C::NX; ++s) {
       mbar_init(&full_x[s], 1);
       mbar_init(&empty_x[s], kIssuers);
     }
-    for (int s = 0; s < C::NA; ++s) mbar_init(&full_a[s], kDqWarps / 2);  // one group
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], kIssuers);  // one MMA commit per issuer
       mbar_init(&acc_empty[b], 4);      // 4 epilogue warps
@@ -574,121 +561,137 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else if (warp == 1 || warp == 14) {
     // ------------------------------------------------------------ MMA issuers
-    // Two threads issue (the issue cost of a tcgen05.mma is mostly per-thread latency):
+    // Two converged warps issue, one elected lane each. An issuing warp touches no shared
+    // memory inside the K loop: after a tcgen05.mma, the next shared-memory access of the
+    // same warp (an mbarrier wait included) stalls until that warp's MMAs have drained,
+    // which at N = 16 costs more than the MMAs themselves. So the dequantisers, which wait
+    // for the activation stage anyway, announce a ready chunk on a named barrier per stage,
+    // and the issuers only bar.sync on it (a named barrier does not stall behind the MMAs).
     // gate/up: issuer i takes matrix i, all K steps; down: issuer i takes the K steps
     // 2i, 2i+1 of every chunk into its own accumulator (the epilogue adds the two).
+    // Every chunk's barrier is met by its dequantiser group, also after a failure (the MMAs
+    // then run on stale operands and the status word carries the error), so the issuers
+    // take every chunk and never wait on a barrier that nobody meets.
     const int iss = (warp == 1) ? 0 : 1;
-    if (lane == 0) {
-      const int mi = GATE_UP ? iss : 0;
-      const int k0 = GATE_UP ? 0 : 2 * iss, k1 = GATE_UP ? kTcBK / 16 : 2 * iss + 2;
-      int it = 0, tile = 0;
-      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
-        const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
-        const int n_mma = (t.nrows + 15) & ~15;
-        const uint32_t idesc = umma_idesc_f16(n_mma);
-        const int b = tile & 1, buse = tile >> 1;
-        if (buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1)) {
-          fail();
-          break;
-        }
-        tc_fence_after();
-        TCT(1, tile, 0);
-        const uint32_t dacc = tmem + b * 128 + iss * kTcNMax;  // this issuer's accumulator
-        bool ok = true;
-        for (int c = 0; c < n_chunks; ++c, ++it) {
-          const int s = it % C::NX;
-          const bool okx = mbar_wait(&full_x[s], (it / C::NX) & 1);
-          TCC(it, 0);
-          const bool oka = okx && mbar_wait(&full_a[s], (it / C::NA) & 1);
-          TCC(it, 1);
-          if (!oka) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // One descriptor and one TMEM address per chunk; the K steps advance them by
-          // constants (32 bytes of B = 2 in the descriptor's address field, 8 columns of A).
-          const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::X_OFF + s * C::XB));
-          const uint32_t at = tmem + C::A_COL0 + s * C::A_COLS + mi * (kTcBK / 2);
-          umma_f16_ts(dacc, at + k0 * 8, bdesc + (uint64_t)(2 * k0), idesc, c > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 1; kk < kTcBK / 16; ++kk)
-            if (k0 + kk < k1)
-              umma_f16_ts_acc(dacc, at + (k0 + kk) * 8, bdesc + (uint64_t)(2 * (k0 + kk)), idesc);
-          umma_commit(&empty_x[s]);  // releases the activation stage and the A stage
-          TCC(it, 2);
-        }
-        if (!ok) {
-          fail();
-          break;
-        }
-        umma_commit(&acc_full[b]);
-        TCT(1, tile, 1);
+    const int mi = GATE_UP ? iss : 0;
+    const int k0 = GATE_UP ? 0 : 2 * iss, k1 = GATE_UP ? kTcBK / 16 : 2 * iss + 2;
+    bool aborted = false;
+    int it = 0, tile = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x, ++tile) {
+      const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
+      const int n_mma = (t.nrows + 15) & ~15;
+      const uint32_t idesc = umma_idesc_f16(n_mma);
+      const int b = tile & 1, buse = tile >> 1;
+      aborted = aborted || *abort_flag;
+      if (!aborted && buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1)) {
+        fail();
+        aborted = true;
       }
-      // all issued MMAs complete before TMEM and shared memory are released
-      umma_commit(drain);
-      mbar_wait(drain, 0);
+      aborted = __any_sync(0xffffffffu, aborted);
+      tc_fence_after();
+      TCT(1, tile, 0);
+      const uint32_t dacc = tmem + b * 128 + iss * kTcNMax;  // this issuer's accumulator
+      for (int c = 0; c < n_chunks; ++c, ++it) {
+        const int s = it % C::NX;
+        named_bar_sync(1 + s, kReadyThreads);
+        tc_fence_after();
+        TCC(it, 1);
+        // One descriptor and one TMEM address per chunk; the K steps advance them by
+        // constants (32 bytes of B = 2 in the descriptor's address field, 8 columns of A).
+        const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::X_OFF + s * C::XB));
+        const uint32_t at = tmem + C::A_COL0 + s * C::A_COLS + mi * (kTcBK / 2);
+#pragma unroll
+        for (int kk = 0; kk < kTcBK / 16; ++kk)
+          if (k0 + kk < k1)
+            umma_f16_ts_warp(dacc, at + (k0 + kk) * 8, bdesc + (uint64_t)(2 * (k0 + kk)), idesc,
+                             (c > 0 || kk > 0) ? 1u : 0u);
+        umma_commit_warp(&empty_x[s]);  // releases the activation stage and the A stage
+        TCC(it, 2);
+      }
+      umma_commit_warp(&acc_full[b]);
+      TCT(1, tile, 1);
     }
+    // all issued MMAs complete before TMEM and shared memory are released
+    umma_commit_warp(drain);
+    mbar_wait(drain, 0);
   } else if (warp < 2 + kDqWarps) {
     // ------------------------------------------------------------ dequantisers
     // Two groups of four warps take alternate chunks (group g: chunks c with c % 2 == g), so
     // two chunks are converted at a time; within a group, warp w covers the weight rows of
-    // TMEM lanes 32 * (w % 4) .. +31 (the lanes a warp may write), both K halves.
+    // TMEM lanes 32 * (w % 4) .. +31 (the lanes a warp may write), both K halves. A group
+    // converts chunk i into A stage i % NA once the MMAs of chunk i - NA have released it,
+    // checks that the chunk's activation stage has landed, and arrives on the chunk's ready
+    // barrier. It arrives for every chunk, also after a failure (then without converting and
+    // without waiting on the producers), and always after the release of the stage: so the
+    // issuers meet each barrier phase exactly once.
     const int r = 32 * (warp & 3) + lane;            // weight row in the tile
     const int group = (warp - 2) >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    bool aborted = false;
     int it = 0, ia = 0, ui = 0;
-    for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++ui) {
+    for (int u = blockIdx.x; u < total; u += gridDim.x, ++ui) {
       const int sbuf = ui & 1;
-      bool ok = true;
+      aborted = aborted || *abort_flag;
       if (threadIdx.x == 64) TCT(2, ui, 0);
-      if constexpr (FMT != 16) ok = mbar_wait(&scale_full[sbuf], (ui >> 1) & 1);
+      if constexpr (FMT != 16) {
+        if (!aborted && !mbar_wait(&scale_full[sbuf], (ui >> 1) & 1)) {
+          fail();
+          aborted = true;
+        }
+      }
+      aborted = __any_sync(0xffffffffu, aborted);
       const uint16_t* sblk = reinterpret_cast<const uint16_t*>(smem + C::S_OFF + sbuf * NM * SL.sb);
-      for (int cw = 0; cw < n_wstages && ok; ++cw, ++it) {
+      for (int cw = 0; cw < n_wstages; ++cw, ++it) {
         const int sw = it % C::NW;
         // every warp waits for every stage before releasing it (keeps the release phases
         // of the stage in order, also for a group with no chunk in it)
-        if (!mbar_wait(&full_w[sw], (it / C::NW) & 1)) {
-          ok = false;
-          break;
+        if (!aborted && !mbar_wait(&full_w[sw], (it / C::NW) & 1)) {
+          fail();
+          aborted = true;
         }
+        aborted = __any_sync(0xffffffffu, aborted);
         const int c_end = min(n_chunks, (cw + 1) * C::SUB);
         for (int c = cw * C::SUB; c < c_end; ++c, ++ia) {
           if ((c & 1) != group) continue;
           const int a = ia % C::NA;
-          float sc[NM];
-#pragma unroll
-          for (int mi = 0; mi < NM; ++mi)
-            sc[mi] = (FMT == 16) ? 1.f
-                                 : bf16_to_f32(sblk[mi * (SL.sb / 2) + r * G + (c * kTcBK) / kGroup]);
-          if (threadIdx.x == 64) TCC(ia, 3);
+          if ((threadIdx.x & 127) == 64) TCC(ia, 3);
+          // the stage's previous chunk is consumed (waited for also after a failure; the
+          // issuers never stop, so this wait ends)
           if (ia >= C::NA && !mbar_wait(&empty_x[a], ((ia / C::NA) - 1) & 1)) {
-            ok = false;
-            break;
+            fail();
+            aborted = true;
           }
-          if (threadIdx.x == 64) TCC(ia, 4);
+          if (!aborted && !mbar_wait(&full_x[a], (ia / C::NX) & 1)) {
+            fail();
+            aborted = true;
+          }
+          aborted = __any_sync(0xffffffffu, aborted);
+          if ((threadIdx.x & 127) == 64) TCC(ia, 4);
+          if (!aborted) {
+            float sc[NM];
 #pragma unroll
-          for (int mi = 0; mi < NM; ++mi) {
-            const uint8_t* raw_row = smem + C::R_OFF + sw * C::WB + mi * C::RAW + r * C::RAW_ROW;
-            uint32_t regs[32];
-            uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[0]);
-            uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[16]);
-            dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 0, sc[mi], lo);
-            dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 1, sc[mi], hi);
-            tmem_st32(lane_base + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2), regs);
+            for (int mi = 0; mi < NM; ++mi)
+              sc[mi] = (FMT == 16) ? 1.f
+                                   : bf16_to_f32(sblk[mi * (SL.sb / 2) + r * G + (c * kTcBK) / kGroup]);
+#pragma unroll
+            for (int mi = 0; mi < NM; ++mi) {
+              const uint8_t* raw_row = smem + C::R_OFF + sw * C::WB + mi * C::RAW + r * C::RAW_ROW;
+              uint32_t regs[32];
+              uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[0]);
+              uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[16]);
+              dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 0, sc[mi], lo);
+              dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 1, sc[mi], hi);
+              tmem_st32(lane_base + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2), regs);
+            }
+            tmem_st_wait();
           }
-          tmem_st_wait();
-          tc_fence_before();  // the stores are complete before the arrive below
+          tc_fence_before();  // the stores are complete before the arrival below
           __syncwarp();
-          if (threadIdx.x == 64) TCC(ia, 5);
-          if (lane == 0) mbar_arrive(&full_a[a]);
+          if ((threadIdx.x & 127) == 64) TCC(ia, 5);
+          named_bar_arrive(1 + a, kReadyThreads);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_w[sw]);  // the stage is read
-      }
-      if (!ok) {
-        fail();
-        break;
       }
       if constexpr (FMT != 16) {
         __syncwarp();
@@ -741,6 +744,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (threadIdx.x == 320) TCT(3, tile, 0);
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + b * 128;
       const int n = t.ntile * kTcM + row;  // output feature
+      // gate/up: where feature n sits in the h row (the K order the down GEMM's bank reads)
+      const int hn = GATE_UP ? k_position(n, interleaved_k(t.shared ? p.shared.fmt : p.routed.fmt)) : n;
       for (int m0 = 0; m0 < t.nrows; m0 += 16) {
         float g[16];
         tmem_ld16(lane_addr + m0, g);
@@ -754,7 +759,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const size_t hrow = (t.shared ? (size_t)p.T * p.k : 0) + t.row0 + m0 + j;
               if (!(fabsf(h) <= 65504.f)) set_status(p.status, DEV_RANGE);
               const __half hh = __float2half_rn(h);
-              p.h[hrow * p.f + n] = *reinterpret_cast<const uint16_t*>(&hh);
+              p.h[hrow * p.f + hn] = *reinterpret_cast<const uint16_t*>(&hh);
             }
           }
         } else {
