@@ -26,10 +26,10 @@
 // fp16 exactly in fp16's range, and q * s rounds once with an 11-bit significand, eight
 // times finer than bf16. Activations and h outside fp16's range set a device status flag.
 // Rings: weights (TMA -> dequant), activations (TMA -> MMA), A (dequant -> MMA, in TMEM;
-// announced on a named barrier per stage), accumulator (MMA -> epilogue, double buffered in
-// TMEM). TMEM columns: accumulators
-// [0, 256) (buffer b: gate at 128 b, up at 128 b + 64), A stages [256, 512). Every wait is bounded; a timeout sets the
-// status word and every role drains and exits (TMEM is freed by its owner).
+// announced on a named barrier per stage), accumulator (MMA -> epilogue, in
+// TMEM). TMEM columns: the accumulator buffers from column 0 (buffer b: gate at 128 b, up at
+// 128 b + 64), then the A stages. Every wait is bounded; a timeout sets the status word and
+// every role drains and exits (TMEM is freed by its owner).
 //
 // Work units (slot, n-tile, m-tile) are ordered with the m-tile fastest, and CTAs take
 // them round-robin, so the m-tiles of one weight tile run at the same time on neighbouring
@@ -53,6 +53,18 @@ __device__ long long g_tct[2][4][16][2];  // [kernel][role][unit][start/end], CT
 __device__ long long g_tcc[2][48][6];  // [kernel][chunk of unit 0][event], CTA 0
 #define TCC(c, ev) \
   do { if (blockIdx.x == 0 && (c) < 48) g_tcc[GATE_UP ? 0 : 1][c][ev] = clock64(); } while (0)
+__device__ long long g_tcw[2][48][8][3];  // [kernel][chunk][dequant warp][start, waited, arrival]
+#define TCW(c, ev) \
+  do { if (blockIdx.x == 0 && lane == 0 && (c) < 48) g_tcw[GATE_UP ? 0 : 1][c][warp - 2][ev] = clock64(); } while (0)
+__device__ long long g_tcs[2][16][8][2];  // [kernel][weight stage][dequant warp][before, after full_w]
+#define TCS(st, ev) \
+  do { if (blockIdx.x == 0 && lane == 0 && (st) < 16) g_tcs[GATE_UP ? 0 : 1][st][warp - 2][ev] = clock64(); } while (0)
+extern "C" __attribute__((visibility("default"))) int moe_tcs_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_tcs, sizeof(g_tcs));
+}
+extern "C" __attribute__((visibility("default"))) int moe_tcw_read(void* dst) {
+  return (int)cudaMemcpyFromSymbol(dst, g_tcw, sizeof(g_tcw));
+}
 extern "C" __attribute__((visibility("default"))) int moe_tcc_read(void* dst) {
   return (int)cudaMemcpyFromSymbol(dst, g_tcc, sizeof(g_tcc));
 }
@@ -62,6 +74,8 @@ extern "C" __attribute__((visibility("default"))) int moe_tct_read(void* dst) {
 #else
 #define TCT(role, ui, se) do {} while (0)
 #define TCC(c, ev) do {} while (0)
+#define TCW(c, ev) do {} while (0)
+#define TCS(st, ev) do {} while (0)
 #endif
 
 constexpr int kTcThreads = 512;  // 16 warps
@@ -80,7 +94,7 @@ struct TcMaps {
   int box_rows[2][kBoxes];      // rows per activation box (16 << box, at most the source's)
 };
 
-template <int FMT, bool GATE_UP> struct TcCfg {
+template <int FMT, bool GATE_UP, int ACC> struct TcCfg {
   static constexpr int NM = GATE_UP ? 2 : 1;
   // A weight stage is 128 bytes of each of 128 rows (one 128-byte swizzle span: full L2
   // lines per row and conflict-free reads), i.e. KW = 256 / 128 / 64 K values for int4 /
@@ -95,10 +109,17 @@ template <int FMT, bool GATE_UP> struct TcCfg {
   static constexpr int WB = NM * RAW;                // weight stage bytes
   static constexpr int W_BUDGET = (GATE_UP ? 128 : 96) * 1024;
   static constexpr int NW = W_BUDGET / WB > 16 ? 16 : W_BUDGET / WB;
-  static constexpr int NX = GATE_UP ? 4 : 6;         // activation stages (= A stages)
+  // TMEM: ACC accumulator buffers of 128 columns (two 64-column accumulators each) from
+  // column 0, then the A stages. One accumulator buffer leaves room for a deeper gate/up A
+  // ring, which lets the dequantisers run ahead of the MMAs; the MMAs of a unit then wait
+  // for the epilogue to have read the previous unit. That pause grows with the unit's rows,
+  // so calls with many rows per expert take two buffers (measured on B200: prefill 523 vs
+  // 578 us with one, a 4096-token call 1232 vs 1322 us with two).
+  static constexpr int ACC_BUFS = ACC;
+  static constexpr int NX = GATE_UP ? (ACC == 1 ? 6 : 4) : 8;  // activation stages (= A stages)
   static constexpr int A_COLS = NM * (kTcBK / 2);    // TMEM columns of one A stage
   static constexpr int NA = NX;                      // A stages in TMEM
-  static constexpr int A_COL0 = 256;
+  static constexpr int A_COL0 = ACC_BUFS * 128;
   static_assert(A_COL0 + NA * A_COLS <= 512, "TMEM budget");
   static_assert(NX <= 15, "one named barrier per stage (ids 1..15)");
   // layout (1024-byte aligned pieces first)
@@ -115,9 +136,9 @@ struct TcSmem {
   int sched_off, bar_off, total;
 };
 
-template <int FMT, bool GATE_UP>
+template <int FMT, bool GATE_UP, int ACC>
 __host__ __device__ inline TcSmem tc_smem(int K, int E) {
-  using C = TcCfg<FMT, GATE_UP>;
+  using C = TcCfg<FMT, GATE_UP, ACC>;
   TcSmem m;
   m.sb = (FMT == 16) ? 0 : kTcM * (K / kGroup) * 2;
   m.sched_off = C::S_OFF + 2 * C::NM * m.sb;
@@ -415,16 +436,16 @@ __device__ __forceinline__ void dequant_half_row(const uint8_t* row, int sw7, in
 
 // ------------------------------------------------------------------ the kernel
 
-template <int FMT, bool GATE_UP>
+template <int FMT, bool GATE_UP, int ACC>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_grouped_kernel(const __grid_constant__ TcMaps maps, Plan p, TcSched S) {
-  using C = TcCfg<FMT, GATE_UP>;
+  using C = TcCfg<FMT, GATE_UP, ACC>;
   constexpr int NM = C::NM;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const TcSmem SL = tc_smem<FMT, GATE_UP>(GATE_UP ? p.d : p.f, p.E);
+  const TcSmem SL = tc_smem<FMT, GATE_UP, ACC>(GATE_UP ? p.d : p.f, p.E);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL.bar_off);
   uint64_t* full_w = bars;                   // [NW]
   uint64_t* empty_w = full_w + C::NW;        // [NW]
@@ -581,7 +602,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
       const int n_mma = (t.nrows + 15) & ~15;
       const uint32_t idesc = umma_idesc_f16(n_mma);
-      const int b = tile & 1, buse = tile >> 1;
+      const int b = tile % C::ACC_BUFS, buse = tile / C::ACC_BUFS;
       aborted = aborted || *abort_flag;
       if (!aborted && buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1)) {
         fail();
@@ -616,14 +637,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_wait(drain, 0);
   } else if (warp < 2 + kDqWarps) {
     // ------------------------------------------------------------ dequantisers
-    // Two groups of four warps take alternate chunks (group g: chunks c with c % 2 == g), so
-    // two chunks are converted at a time; within a group, warp w covers the weight rows of
-    // TMEM lanes 32 * (w % 4) .. +31 (the lanes a warp may write), both K halves. A group
-    // converts chunk i into A stage i % NA once the MMAs of chunk i - NA have released it,
-    // checks that the chunk's activation stage has landed, and arrives on the chunk's ready
-    // barrier. It arrives for every chunk, also after a failure (then without converting and
-    // without waiting on the producers), and always after the release of the stage: so the
-    // issuers meet each barrier phase exactly once.
+    // Two groups of four warps take alternate steps of CH consecutive chunks (group g: steps
+    // j of a unit with j % 2 == g), so two steps are converted at a time; within a group, warp
+    // w covers the weight rows of TMEM lanes 32 * (w % 4) .. +31 (the lanes a warp may
+    // write), both K halves. A group converts chunk i into A stage i % NA once the MMAs of
+    // chunk i - NA have released it, checks that the chunk's activation stage has landed, and
+    // arrives on the chunk's ready barrier. Two chunks a step halve the fixed cost of the
+    // waits, the store wait and the arrivals per chunk. A group arrives for every chunk, also
+    // after a failure (then without converting and without waiting on the producers), and
+    // always after the release of the stage: so the issuers meet each barrier phase exactly
+    // once.
+    constexpr int CH = C::SUB >= 2 ? 2 : 1;  // chunks a step (K is a multiple of 128)
     const int r = 32 * (warp & 3) + lane;            // weight row in the tile
     const int group = (warp - 2) >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
@@ -645,50 +669,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int sw = it % C::NW;
         // every warp waits for every stage before releasing it (keeps the release phases
         // of the stage in order, also for a group with no chunk in it)
+        TCS(it, 0);
         if (!aborted && !mbar_wait(&full_w[sw], (it / C::NW) & 1)) {
           fail();
           aborted = true;
         }
         aborted = __any_sync(0xffffffffu, aborted);
+        TCS(it, 1);
         const int c_end = min(n_chunks, (cw + 1) * C::SUB);
-        for (int c = cw * C::SUB; c < c_end; ++c, ++ia) {
-          if ((c & 1) != group) continue;
-          const int a = ia % C::NA;
+        for (int c = cw * C::SUB; c < c_end; c += CH, ia += CH) {
+          if (((c / CH) & 1) != group) continue;
           if ((threadIdx.x & 127) == 64) TCC(ia, 3);
-          // the stage's previous chunk is consumed (waited for also after a failure; the
-          // issuers never stop, so this wait ends)
-          if (ia >= C::NA && !mbar_wait(&empty_x[a], ((ia / C::NA) - 1) & 1)) {
-            fail();
-            aborted = true;
-          }
-          if (!aborted && !mbar_wait(&full_x[a], (ia / C::NX) & 1)) {
-            fail();
-            aborted = true;
+          TCW(ia, 0);
+#pragma unroll
+          for (int j = 0; j < CH; ++j) {
+            const int a = (ia + j) % C::NA;
+            // the stage's previous chunk is consumed (waited for also after a failure; the
+            // issuers never stop, so this wait ends)
+            if (ia + j >= C::NA && !mbar_wait(&empty_x[a], (((ia + j) / C::NA) - 1) & 1)) {
+              fail();
+              aborted = true;
+            }
+            if (!aborted && !mbar_wait(&full_x[a], ((ia + j) / C::NX) & 1)) {
+              fail();
+              aborted = true;
+            }
           }
           aborted = __any_sync(0xffffffffu, aborted);
           if ((threadIdx.x & 127) == 64) TCC(ia, 4);
+          TCW(ia, 1);
           if (!aborted) {
-            float sc[NM];
 #pragma unroll
-            for (int mi = 0; mi < NM; ++mi)
-              sc[mi] = (FMT == 16) ? 1.f
-                                   : bf16_to_f32(sblk[mi * (SL.sb / 2) + r * G + (c * kTcBK) / kGroup]);
+            for (int j = 0; j < CH; ++j) {
+              const int a = (ia + j) % C::NA, cc = c + j;
 #pragma unroll
-            for (int mi = 0; mi < NM; ++mi) {
-              const uint8_t* raw_row = smem + C::R_OFF + sw * C::WB + mi * C::RAW + r * C::RAW_ROW;
-              uint32_t regs[32];
-              uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[0]);
-              uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[16]);
-              dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 0, sc[mi], lo);
-              dequant_half_row<FMT>(raw_row, r & 7, c - cw * C::SUB, 1, sc[mi], hi);
-              tmem_st32(lane_base + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2), regs);
+              for (int mi = 0; mi < NM; ++mi) {
+                const float sc = (FMT == 16) ? 1.f
+                                 : bf16_to_f32(sblk[mi * (SL.sb / 2) + r * G + (cc * kTcBK) / kGroup]);
+                const uint8_t* raw_row = smem + C::R_OFF + sw * C::WB + mi * C::RAW + r * C::RAW_ROW;
+                uint32_t regs[32];
+                uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[0]);
+                uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&regs[16]);
+                dequant_half_row<FMT>(raw_row, r & 7, cc - cw * C::SUB, 0, sc, lo);
+                dequant_half_row<FMT>(raw_row, r & 7, cc - cw * C::SUB, 1, sc, hi);
+                tmem_st32(lane_base + C::A_COL0 + a * C::A_COLS + mi * (kTcBK / 2), regs);
+              }
             }
             tmem_st_wait();
           }
-          tc_fence_before();  // the stores are complete before the arrival below
+          tc_fence_before();  // the stores are complete before the arrivals below
           __syncwarp();
           if ((threadIdx.x & 127) == 64) TCC(ia, 5);
-          named_bar_arrive(1 + a, kReadyThreads);
+          TCW(ia, 2);
+#pragma unroll
+          for (int j = 0; j < CH; ++j) named_bar_arrive(1 + (ia + j) % C::NA, kReadyThreads);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_w[sw]);  // the stage is read
@@ -735,8 +769,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int tile = 0;
     for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
       const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
-      const int b = tile & 1;
-      if (!mbar_wait(&acc_full[b], (tile >> 1) & 1)) {
+      const int b = tile % C::ACC_BUFS;
+      if (!mbar_wait(&acc_full[b], (tile / C::ACC_BUFS) & 1)) {
         fail();
         break;
       }
@@ -840,10 +874,10 @@ TcSched tc_sched_view(void* base, int E) {
   return s;
 }
 
-template <int FMT, bool GATE_UP>
+template <int FMT, bool GATE_UP, int ACC>
 static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t* xg,
                                  cudaStream_t st) {
-  using C = TcCfg<FMT, GATE_UP>;
+  using C = TcCfg<FMT, GATE_UP, ACC>;
   const int K = GATE_UP ? p.d : p.f;
   const int N = GATE_UP ? p.f : p.d;
   const int wbytes_per_row = K * FMT / 8;  // int4: K/2, int8: K, bf16: 2K
@@ -886,8 +920,8 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
         return cudaErrorInvalidValue;
     }
   }
-  auto kern = tc_grouped_kernel<FMT, GATE_UP>;
-  const int smem = tc_smem<FMT, GATE_UP>(K, p.E).total;
+  auto kern = tc_grouped_kernel<FMT, GATE_UP, ACC>;
+  const int smem = tc_smem<FMT, GATE_UP, ACC>(K, p.E).total;
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -913,13 +947,13 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
   return cudaLaunchKernelEx(&cfg, kern, maps, p, S);
 }
 
-template <bool GATE_UP>
+template <bool GATE_UP, int ACC>
 static cudaError_t launch_tc(const Plan& p, const TcSched& S, const uint16_t* xg,
                              cudaStream_t st) {
   switch (p.routed.fmt) {
-    case 4: return launch_tc_fmt<4, GATE_UP>(p, S, xg, st);
-    case 8: return launch_tc_fmt<8, GATE_UP>(p, S, xg, st);
-    default: return launch_tc_fmt<16, GATE_UP>(p, S, xg, st);
+    case 4: return launch_tc_fmt<4, GATE_UP, ACC>(p, S, xg, st);
+    case 8: return launch_tc_fmt<8, GATE_UP, ACC>(p, S, xg, st);
+    default: return launch_tc_fmt<16, GATE_UP, ACC>(p, S, xg, st);
   }
 }
 
@@ -943,12 +977,14 @@ cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaSt
   return cudaLaunchKernelEx(&cfg, tc_prep_kernel, p, S, xg);
 }
 
+// Gate/up with two accumulator buffers when the routed experts average 32 rows or more.
 cudaError_t launch_tc_gate_up(const Plan& p, const TcSched& S, const uint16_t* xg,
                               cudaStream_t st) {
-  return launch_tc<true>(p, S, xg, st);
+  if ((long long)p.T * p.k >= 32LL * p.E) return launch_tc<true, 2>(p, S, xg, st);
+  return launch_tc<true, 1>(p, S, xg, st);
 }
 cudaError_t launch_tc_down(const Plan& p, const TcSched& S, cudaStream_t st) {
-  return launch_tc<false>(p, S, nullptr, st);
+  return launch_tc<false, 2>(p, S, nullptr, st);
 }
 
 }  // namespace moe

@@ -215,6 +215,16 @@ def test_tc_formats_small(B, fmt, shared):
     check_layer(B, B.DeviceLayer(L), L, L.x, "tc")
 
 
+@pytest.mark.parametrize("fmt", ["int4", "int8", "bf16"])
+def test_tc_formats_many_rows_per_expert(B, fmt):
+    """32+ rows per routed expert on average: the gate/up GEMM's two-accumulator layout."""
+    cfg = synth.LayerConfig(f"tc-wide-{fmt}", T=160, d=384, E=6, k=2, f=256, n_shared=1,
+                            fmt=fmt, seed=17)
+    assert cfg.T * cfg.k >= 32 * cfg.E
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "tc")
+
+
 def test_tc_tiny(B, tiny):
     L, dl = tiny
     check_layer(B, dl, L, L.x, "tc")
