@@ -62,18 +62,32 @@ __device__ int block_exclusive_scan(int v, int* total) {
   return base + incl - v;
 }
 
-// Pass 2: one 1024-thread CTA. Per expert: counts over chunks -> per-chunk bases; then the
-// exclusive scan over experts; then the active-expert list.
+// Pass 2: one 1024-thread CTA. Per expert: counts over chunks -> per-chunk bases within the
+// expert (the scatter adds the expert's offset); then the exclusive scan over experts; then
+// the active-expert list. The chunk counts are loaded 16 at a time (independent loads; only
+// the running sum is serial), which keeps the pass from running at one L2 round trip a chunk.
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ cta_hist,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ active,
                                                          int n_chunks, int E) {
+  constexpr int kBatch = 16;
   const int e = threadIdx.x;
   int cnt = 0;
   if (e < E) {
-    for (int c = 0; c < n_chunks; ++c) {
+    int c = 0;
+    for (; c + kBatch <= n_chunks; c += kBatch) {
+      int h[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) h[j] = cta_hist[(size_t)(c + j) * E + e];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        cta_hist[(size_t)(c + j) * E + e] = cnt;  // exclusive base within the expert
+        cnt += h[j];
+      }
+    }
+    for (; c < n_chunks; ++c) {
       const int h = cta_hist[(size_t)c * E + e];
-      cta_hist[(size_t)c * E + e] = cnt;  // exclusive base within the expert
+      cta_hist[(size_t)c * E + e] = cnt;
       cnt += h;
     }
   }
@@ -84,7 +98,6 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
   const int apos = block_exclusive_scan(flag, &n_active);
   if (e < E) {
     offsets[e] = off;
-    for (int c = 0; c < n_chunks; ++c) cta_hist[(size_t)c * E + e] += off;
     if (flag) active[1 + apos] = e;
   }
   if (e == 0) {
@@ -95,15 +108,17 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
 
 // Pass 3: each 32-thread CTA walks its chunk in order, 32 assignments at a time; inside a
 // step, lanes with the same expert are ranked by lane (match_any), and a per-expert running
-// position in shared memory carries the order across steps.
+// position in shared memory (the expert's offset + the chunk's base within the expert)
+// carries the order across steps.
 __global__ void __launch_bounds__(32) perm_scatter_kernel(const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ cta_base,
+                                                          const int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ perm,
                                                           int32_t* __restrict__ inv, int n,
                                                           int E) {
   extern __shared__ int32_t run[];
   const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) run[e] = cta_base[(size_t)blockIdx.x * E + e];
+  for (int e = lane; e < E; e += 32) run[e] = offsets[e] + cta_base[(size_t)blockIdx.x * E + e];
   __syncwarp();
   const int a0 = blockIdx.x * kPermChunk;
   for (int s = 0; s < kPermChunk; s += 32) {
@@ -202,7 +217,8 @@ cudaError_t launch_permute(const Plan& p, cudaStream_t st) {
   const size_t smem = sizeof(int32_t) * p.E;
   perm_hist_kernel<<<chunks, 32, smem, st>>>(p.topk_idx, p.cta_hist, n, p.E, p.status);
   perm_scan_kernel<<<1, 1024, 0, st>>>(p.cta_hist, p.offsets, p.active, chunks, p.E);
-  perm_scatter_kernel<<<chunks, 32, smem, st>>>(p.topk_idx, p.cta_hist, p.perm, p.inv, n, p.E);
+  perm_scatter_kernel<<<chunks, 32, smem, st>>>(p.topk_idx, p.cta_hist, p.offsets, p.perm, p.inv,
+                                                 n, p.E);
   return cudaGetLastError();
 }
 

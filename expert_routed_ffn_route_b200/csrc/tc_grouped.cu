@@ -335,8 +335,10 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
     const int rows = n + (p.has_shared ? p.T : 0);
     const int chunks = p.d / 8;
     bool range_ok = true;
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < (size_t)rows * chunks;
-         i += (size_t)gridDim.x * blockDim.x) {
+    const size_t total = (size_t)rows * chunks, stride = (size_t)gridDim.x * blockDim.x;
+    // four independent 16-byte pieces in flight per thread and iteration
+#pragma unroll 4
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
       const int r = (int)(i / chunks), c = (int)(i % chunks);
       const int t = (r < n) ? p.perm[r] / p.k : r - n;
       const bool il = interleaved_k((r < n) ? p.routed.fmt : p.shared.fmt);
