@@ -154,7 +154,7 @@ struct Plan {
   float* y_assign;     // [T*k*d]
   float* y_shared;     // [T*d]
   int32_t* status;
-  int32_t* ticket;     // zero between calls; the fused routing kernel's completion counter
+  int32_t* ticket;     // [2], zero between calls: the fused routing kernel's arrival counters
   uint32_t* gbar;      // grid-barrier word of the single-kernel 1-token path (any value)
   int32_t* tile_cnt;   // [d / 16] per-output-tile arrival counters, zero between calls
   uint16_t* xg;        // tensor-core path: fp16 x rows in grouped order, then the shared
@@ -175,7 +175,7 @@ struct TcSched {
 };
 
 // The synchronisation block at the start of the workspace: status word (offset 0), routing
-// ticket (16), grid-barrier word (32), then one arrival counter per 16-row output tile (256).
+// tickets (16, 20), grid-barrier word (32), then one arrival counter per 16-row output tile (256).
 inline size_t sync_bytes(int d) { return 256 + (size_t)4 * (d / 16); }
 
 // Permutation chunking (assignments per scatter CTA).

@@ -3,14 +3,17 @@
 //
 // Phase 1 (all CTAs): router logits l[t][e] = x_t . Wr_e (+ b_e) in fp32, one warp per
 // expert row, 128-bit loads, every token of the call against the row while it is in
-// registers. Phase 2 (the last CTA to finish phase 1, found with an atomic ticket after a
-// memory fence; nobody waits): per token the stable top-k and the gates, then the
-// expert-major plan and the active-expert list. The ticket is reset for the next call.
+// registers. Phase 2 (CTAs 0 .. T-1, once every CTA has counted itself in a ticket after a
+// memory fence): CTA t ranks token t (stable top-k and gates). Phase 3 (the last of those to
+// finish, found with a second ticket): the expert-major plan and the active-expert list,
+// then both tickets are cleared for the next call.
 //
 // Rules followed: deterministic stable top-k, ties to the lower expert index
 // (Qwen3.8-Flash-Next-Dual-GPU README, "Independent decode lane"); gates = softmax over the
 // selected logits; plan = counts, exclusive scan, stable scatter (README, "Dedicated
 // prefill lane", step 1).
+#include <algorithm>
+
 #include "pipeline.cuh"
 
 namespace moe {
@@ -38,9 +41,10 @@ extern "C" __attribute__((visibility("default"))) int moe_rtrace_read(void* dst)
 constexpr int kRFWarps = 4;
 constexpr int kRFThreads = 32 * kRFWarps;
 constexpr int kRFMaxT = 32;
+static_assert(kRFMaxT % 2 == 0, "the logits take tokens two at a time");
 
 __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t* ticket) {
-  __shared__ int s_last;  // CTA 0: all other CTAs arrived
+  __shared__ int s_last;  // this CTA ranked the last token: it builds the plan
   __shared__ int s_idx[kRFMaxT * kMaxK];
   __shared__ int s_cnt[kMaxE];
   __shared__ int s_off[kMaxE + 1];
@@ -61,8 +65,10 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
 
   // ---------------------------------------------------------------- logits
   // A lane owns 16-byte pieces c = lane + 32 i of the router row (d <= 8192: i < 32); the
-  // row is loaded in batches of 8 pieces, all in flight together, then every token is
-  // applied to the batch while it sits in registers.
+  // row is loaded in batches of 8 pieces, all in flight together, then the tokens are applied
+  // to the batch two at a time while it sits in registers: both tokens' 16 loads are issued
+  // before their products (the second row index is clamped, so the loads need no guard; a
+  // product past the last token is never written).
   const int n16 = d / 8;
   for (int e = blockIdx.x * kRFWarps + warp; e < E; e += gridDim.x * kRFWarps) {
     const uint4* wrow = reinterpret_cast<const uint4*>(p.router_w + (size_t)e * d);
@@ -78,24 +84,30 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
         wv[i] = (c < n16) ? __ldg(wrow + c) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int t = 0; t < kRFMaxT; ++t) {
-        if (t >= T) break;
-        const uint4* xrow = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
-        uint4 xv[8];
+      for (int t0 = 0; t0 < kRFMaxT; t0 += 2) {
+        if (t0 >= T) break;
+        const int t1 = min(t0 + 1, T - 1);
+        const uint4* xa_row = reinterpret_cast<const uint4*>(p.x + (size_t)t0 * d);
+        const uint4* xb_row = reinterpret_cast<const uint4*>(p.x + (size_t)t1 * d);
+        uint4 xa[8], xb[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int c = c0 + lane + 32 * i;
-          xv[i] = (c < n16) ? __ldg(xrow + c) : make_uint4(0, 0, 0, 0);
+          xa[i] = (c < n16) ? __ldg(xa_row + c) : make_uint4(0, 0, 0, 0);
+          xb[i] = (c < n16) ? __ldg(xb_row + c) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
-          const uint32_t xx[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+          const uint32_t aa[4] = {xa[i].x, xa[i].y, xa[i].z, xa[i].w};
+          const uint32_t bb[4] = {xb[i].x, xb[i].y, xb[i].z, xb[i].w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            acc[t] = fmaf(__uint_as_float(xx[q] << 16), __uint_as_float(ww[q] << 16), acc[t]);
-            acc[t] = fmaf(__uint_as_float(xx[q] & 0xffff0000u),
-                          __uint_as_float(ww[q] & 0xffff0000u), acc[t]);
+            const float w0 = __uint_as_float(ww[q] << 16), w1 = __uint_as_float(ww[q] & 0xffff0000u);
+            acc[t0] = fmaf(__uint_as_float(aa[q] << 16), w0, acc[t0]);
+            acc[t0] = fmaf(__uint_as_float(aa[q] & 0xffff0000u), w1, acc[t0]);
+            acc[t0 + 1] = fmaf(__uint_as_float(bb[q] << 16), w0, acc[t0 + 1]);
+            acc[t0 + 1] = fmaf(__uint_as_float(bb[q] & 0xffff0000u), w1, acc[t0 + 1]);
           }
         }
       }
@@ -110,67 +122,66 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
     }
   }
 
-  // ---------------------------------------------------------------- ticket
-  // CTAs 1.. publish their logits and leave; CTA 0 (always the same one, so the SM that
-  // runs the serial tail below keeps its code in the instruction cache from call to call)
-  // waits, boundedly, until all of them have arrived. All CTAs of this grid are resident
-  // together (gridDim <= E / 4 <= 256, one or two small CTAs per SM).
+  // ---------------------------------------------------------------- tickets
+  // Every CTA publishes its logits and counts itself in ticket[0]; CTAs T.. leave. CTA t < T
+  // waits, boundedly, until all CTAs have counted themselves (all CTAs of this grid are
+  // resident together: gridDim = max(E / 4, T) <= 256 small CTAs), ranks token
+  // t, and counts itself in ticket[1]; the last one builds the plan. After a timeout the
+  // status word is set and the CTA goes on (its picks are then unreliable, but every ticket
+  // is still met and cleared).
   RTRACE(1);
   __threadfence();
   __syncthreads();
-  if (blockIdx.x != 0) {
-    if (threadIdx.x == 0) atomicAdd(ticket, 1);
+  if (threadIdx.x == 0) atomicAdd(&ticket[0], 1);
+  if ((int)blockIdx.x >= T) {
     if (threadIdx.x == 0) KT_EXIT(0);
     return;  // an exited CTA counts as having released its dependents
   }
   if (threadIdx.x == 0) {
     const long long t0 = clock64();
-    int seen = 0;
-    while ((seen = *(volatile int*)ticket) < (int)gridDim.x - 1) {
+    while (*(volatile int*)&ticket[0] < (int)gridDim.x) {
       if (clock64() - t0 > kWaitCycles) {
         set_status(p.status, DEV_TIMEOUT);
         break;
       }
     }
-    s_last = (seen >= (int)gridDim.x - 1);
   }
   __syncthreads();
   RTRACE(2);
-  if (!s_last) {  // timed out: leave the outputs untouched; the status word says why
-    if (threadIdx.x == 0) *ticket = 0;
-    pdl_trigger();
-    return;
-  }
   __threadfence();
 #ifdef MOE_TRACE
   long long c_fence = clock64();
 #endif
 
   // ---------------------------------------------------------------- top-k and gates
-  for (int t = warp; t < T; t += kRFWarps) {
+  if (warp == 0) {
+    const int t = blockIdx.x;
     int e;
     uint32_t key;
-#ifdef MOE_TRACE
-    long long c_a = clock64();
-#endif
     warp_topk(p.logits + (size_t)t * E, E, k, lane, &e, &key);
-#ifdef MOE_TRACE
-    if (t == 0 && lane == 0) { g_ktime[7][0] = c_a - c_fence; g_ktime[7][1] = clock64() - c_fence; }
-#endif
     const uint32_t top = __shfl_sync(0xffffffffu, key, 0);
     const float g = warp_topk_gate(key, top, k, lane);
     if (lane < k) {
       p.topk_idx[(size_t)t * k + lane] = e;
       p.topk_w[(size_t)t * k + lane] = g;
-      s_idx[t * k + lane] = e;
     }
-    __syncwarp();
   }
-  __syncthreads();
   RTRACE(3);
 #ifdef MOE_TRACE
   if (threadIdx.x == 0) g_ktime[5][1] = clock64() - c_fence;
 #endif
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&ticket[1], 1) == T - 1);
+  __syncthreads();
+  if (!s_last) {
+    if (threadIdx.x == 0) KT_EXIT(0);
+    return;
+  }
+  __threadfence();
+  for (int a = threadIdx.x; a < T * k; a += kRFThreads) s_idx[a] = __ldcg(p.topk_idx + a);
+  __syncthreads();
+
   // ---------------------------------------------------------------- plan
   const int n = T * k;
   if (n <= 32) {
@@ -268,7 +279,10 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
   if (threadIdx.x == 0) g_ktime[6][0] = clock64() - c_fence;
 #endif
   __syncthreads();
-  if (threadIdx.x == 0) *ticket = 0;
+  if (threadIdx.x == 0) {
+    ticket[0] = 0;
+    ticket[1] = 0;
+  }
   // The next kernel is released only now: kernels whose CTAs wait early for this one share
   // the SMs and slow the last CTA down.
   pdl_trigger();
@@ -277,8 +291,9 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
 
 bool route_fused_supported(const Plan& p) { return p.T <= kRFMaxT && p.E <= kMaxE; }
 
+// One CTA per 4 expert rows and at least one per token (CTA t ranks token t).
 cudaError_t launch_route_fused(const Plan& p, int32_t* ticket, cudaStream_t st) {
-  const int blocks = (p.E + kRFWarps - 1) / kRFWarps;
+  const int blocks = std::max((p.E + kRFWarps - 1) / kRFWarps, p.T);
   route_fused_kernel<<<blocks, kRFThreads, 0, st>>>(p, ticket);
   return cudaGetLastError();
 }

@@ -118,7 +118,9 @@ MOE_API moe_status moe_validate(const moe_layer* L);
 
 /* Bytes of device workspace every call on this layer needs (0 if L is invalid).
  * The workspace is caller-owned, 256-byte aligned, and may be reused between calls
- * that are ordered on one stream; concurrent calls need separate workspaces. */
+ * that are ordered on one stream; concurrent calls need separate workspaces. Fill it with
+ * zeros before its first use (cudaMemset): the calls keep the counters at its start at zero
+ * from one call to the next. */
 MOE_API size_t moe_workspace_size(const moe_layer* L);
 
 /* Route: topk_idx int32 [T][k] (expert ids, rank order) and topk_w fp32 [T][k]
