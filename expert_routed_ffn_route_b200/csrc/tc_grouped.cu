@@ -331,33 +331,36 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
     }
   }
   {
+    // one row per warp, lanes over the row's 16-byte pieces: the source token and the K order
+    // are worked out once per row
     const int n = p.T * p.k;
     const int rows = n + (p.has_shared ? p.T : 0);
     const int chunks = p.d / 8;
+    const int warps = blockDim.x / 32, lane = threadIdx.x & 31;
     bool range_ok = true;
-    const size_t total = (size_t)rows * chunks, stride = (size_t)gridDim.x * blockDim.x;
-    // four independent 16-byte pieces in flight per thread and iteration
-#pragma unroll 4
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-      const int r = (int)(i / chunks), c = (int)(i % chunks);
+    for (int r = blockIdx.x * warps + (int)(threadIdx.x >> 5); r < rows; r += gridDim.x * warps) {
       const int t = (r < n) ? p.perm[r] / p.k : r - n;
       const bool il = interleaved_k((r < n) ? p.routed.fmt : p.shared.fmt);
-      const uint4 v = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d)[c];
-      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-      float e[8];  // K values 8c .. 8c+7
+      const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d);
+      uint4* dst = reinterpret_cast<uint4*>(xg + (size_t)r * p.d);
+      for (int c = lane; c < chunks; c += 32) {
+        const uint4 v = src[c];
+        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+        float e[8];  // K values 8c .. 8c+7
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        e[2 * q] = __uint_as_float(vv[q] << 16);
-        e[2 * q + 1] = __uint_as_float(vv[q] & 0xffff0000u);
-        range_ok &= (fabsf(e[2 * q]) <= 65504.f) && (fabsf(e[2 * q + 1]) <= 65504.f);
-      }
-      uint32_t o[4];
+        for (int q = 0; q < 4; ++q) {
+          e[2 * q] = __uint_as_float(vv[q] << 16);
+          e[2 * q + 1] = __uint_as_float(vv[q] & 0xffff0000u);
+          range_ok &= (fabsf(e[2 * q]) <= 65504.f) && (fabsf(e[2 * q + 1]) <= 65504.f);
+        }
+        uint32_t o[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        __half2 h = il ? __floats2half2_rn(e[q], e[q + 4]) : __floats2half2_rn(e[2 * q], e[2 * q + 1]);
-        o[q] = *reinterpret_cast<uint32_t*>(&h);
+        for (int q = 0; q < 4; ++q) {
+          __half2 h = il ? __floats2half2_rn(e[q], e[q + 4]) : __floats2half2_rn(e[2 * q], e[2 * q + 1]);
+          o[q] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
       }
-      reinterpret_cast<uint4*>(xg + (size_t)r * p.d)[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (!range_ok) set_status(p.status, DEV_RANGE);
   }
@@ -965,8 +968,8 @@ bool tc_supported(const Plan& p) {
 }
 
 cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st) {
-  const long long work = ((long long)p.T * p.k + p.T) * (p.d / 8);
-  const int blocks = (int)std::max(1LL, std::min<long long>(1184, (work + 255) / 256));
+  const long long rows = (long long)p.T * p.k + p.T;  // one warp a row, 8 rows a CTA
+  const int blocks = (int)std::max(1LL, std::min<long long>(1184, (rows + 7) / 8));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(256);
