@@ -41,18 +41,22 @@ struct Unit {
   int tile;       // 32-row tile of the weight matrix
 };
 
-__device__ __forceinline__ bool get_unit(const Plan& p, int u, int n_tiles, Unit& out) {
+// part: 0 both banks, 1 the routed bank only, 2 the shared expert only (one launch per bank
+// when the two banks have different formats).
+__device__ __forceinline__ bool get_unit(const Plan& p, int u, int n_tiles, int part, Unit& out) {
   const int n_active = p.active[0];
+  if (part == 2) u += n_active * n_tiles;  // skip the routed slots
   const int slot = u / n_tiles;
   out.tile = u % n_tiles;
   if (slot < n_active) {
+    if (part == 2) return false;
     out.e = p.active[1 + slot];
     out.shared = false;
     out.row_begin = p.offsets[out.e];
     out.nrows = p.offsets[out.e + 1] - out.row_begin;
     return true;
   }
-  if (slot == n_active && p.has_shared) {
+  if (slot == n_active && p.has_shared && part != 1) {
     out.e = 0;
     out.shared = true;
     out.row_begin = 0;
@@ -65,7 +69,7 @@ __device__ __forceinline__ bool get_unit(const Plan& p, int u, int n_tiles, Unit
 // GATE_UP: weights gate+up [f][d], activations x (gathered by perm), output h (bf16).
 // !GATE_UP: weights down [d][f], activations h, output y (fp32).
 template <int FMT, bool GATE_UP>
-__global__ void __launch_bounds__(kThreads) gemv_ffn_kernel(Plan p) {
+__global__ void __launch_bounds__(kThreads) gemv_ffn_kernel(Plan p, int part) {
   constexpr int NM = GATE_UP ? 2 : 1;
   constexpr int U = FmtInfo<FMT>::U;
   constexpr int PF = (FMT == 4) ? 5 : (FMT == 8 ? (GATE_UP ? 3 : 4) : 2);
@@ -88,7 +92,7 @@ __global__ void __launch_bounds__(kThreads) gemv_ffn_kernel(Plan p) {
 
   for (int u = blockIdx.x;; u += gridDim.x) {
     Unit un;
-    if (!get_unit(p, u, n_tiles, un)) break;
+    if (!get_unit(p, u, n_tiles, part, un)) break;
     const Bank& bank = un.shared ? p.shared : p.routed;
     const int ra_row = un.tile * kRowsCTA + rt * 16 + grp;
     const int rb_row = ra_row + 8;
@@ -213,7 +217,7 @@ struct LaunchCache {
 };
 
 template <int FMT, bool GATE_UP>
-static cudaError_t launch_one(const Plan& p, cudaStream_t st) {
+static cudaError_t launch_one(const Plan& p, int part, cudaStream_t st) {
   const int K = GATE_UP ? p.d : p.f;
   const int N = GATE_UP ? p.f : p.d;
   const int NM = GATE_UP ? 2 : 1;
@@ -241,21 +245,32 @@ static cudaError_t launch_one(const Plan& p, cudaStream_t st) {
     per_sm = std::max(1, cache.per_sm);
     sms = cache.sms;
   }
-  const int max_slots = std::min(p.E, p.T * p.k) + (p.has_shared ? 1 : 0);
+  const int routed_slots = std::min(p.E, p.T * p.k), shared_slots = p.has_shared ? 1 : 0;
+  const int max_slots = part == 1 ? routed_slots
+                                  : (part == 2 ? shared_slots : routed_slots + shared_slots);
   const long long units = (long long)max_slots * (N / kRowsCTA);
   const int grid = (int)std::max(1LL, std::min<long long>(units, (long long)per_sm * sms));
-  kern<<<grid, kThreads, smem, st>>>(p);
+  kern<<<grid, kThreads, smem, st>>>(p, part);
   return cudaGetLastError();
 }
 
 template <bool GATE_UP>
-static cudaError_t launch_fmt(const Plan& p, cudaStream_t st) {
-  // both banks share one format (checked on the host)
-  switch (p.routed.fmt) {
-    case 4: return launch_one<4, GATE_UP>(p, st);
-    case 8: return launch_one<8, GATE_UP>(p, st);
-    default: return launch_one<16, GATE_UP>(p, st);
+static cudaError_t launch_part(const Plan& p, int fmt, int part, cudaStream_t st) {
+  switch (fmt) {
+    case 4: return launch_one<4, GATE_UP>(p, part, st);
+    case 8: return launch_one<8, GATE_UP>(p, part, st);
+    default: return launch_one<16, GATE_UP>(p, part, st);
   }
+}
+
+// One launch for both banks when they share a format; otherwise the routed experts and the
+// shared expert in two launches, each with its own format.
+template <bool GATE_UP>
+static cudaError_t launch_fmt(const Plan& p, cudaStream_t st) {
+  if (!p.has_shared || p.shared.fmt == p.routed.fmt) return launch_part<GATE_UP>(p, p.routed.fmt, 0, st);
+  const cudaError_t err = launch_part<GATE_UP>(p, p.routed.fmt, 1, st);
+  if (err != cudaSuccess) return err;
+  return launch_part<GATE_UP>(p, p.shared.fmt, 2, st);
 }
 
 cudaError_t launch_gemv_gate_up(const Plan& p, cudaStream_t st) { return launch_fmt<true>(p, st); }

@@ -357,7 +357,7 @@ extern "C" __attribute__((visibility("default"))) int moe_trace_read(void* dst) 
 #endif
 
 bool tma_gemv_supported(const Plan& p) {
-  if (p.routed.fmt != 4) return false;
+  if (p.routed.fmt != 4 || (p.has_shared && p.shared.fmt != 4)) return false;
   return tma_smem_layout<true>(p.d).total <= 227 * 1024 &&
          tma_smem_layout<false>(p.f).total <= 227 * 1024;
 }

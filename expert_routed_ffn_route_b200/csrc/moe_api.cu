@@ -45,7 +45,6 @@ moe_status validate(const moe_layer* L) {
   if (!bank_ok(L->routed, L->E, L->d, L->f)) return MOE_ERR_INVALID_ARG;
   if (L->shared.n_exp != 0 && L->shared.n_exp != 1) return MOE_ERR_UNSUPPORTED;
   if (!bank_ok(L->shared, L->shared.n_exp, L->d, L->f)) return MOE_ERR_INVALID_ARG;
-  if (L->shared.n_exp == 1 && L->shared.fmt != L->routed.fmt) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -382,8 +381,9 @@ int32_t moe_launches_per_call(const moe_layer* L) {
   }
   if (use_fused(p)) return 1;
   const int route = route_fused_supported(p) ? 1 : (2 + (L->T * L->k <= 1024 ? 1 : 3));
-  const int ffn = use_tc(p) ? 3 : 2;  // (+ gather/schedule) gate/up, down
-  return route + ffn + 1;             // + combine
+  int ffn = use_tc(p) ? 3 : 2;  // (+ gather/schedule) gate/up, down
+  if (p.has_shared && p.shared.fmt != p.routed.fmt) ffn += 2;  // each GEMM once per bank
+  return route + ffn + 1;       // + combine
 }
 
 moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,

@@ -443,7 +443,7 @@ __device__ __forceinline__ void dequant_half_row(const uint8_t* row, int sw7, in
 
 template <int FMT, bool GATE_UP, int ACC>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_grouped_kernel(const __grid_constant__ TcMaps maps, Plan p, TcSched S) {
+    tc_grouped_kernel(const __grid_constant__ TcMaps maps, Plan p, TcSched S, int part) {
   using C = TcCfg<FMT, GATE_UP, ACC>;
   constexpr int NM = C::NM;
   extern __shared__ uint8_t smem_raw[];
@@ -523,7 +523,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   __syncthreads();
-  const int total = Ss.mt_prefix[n_slots] * n_tiles;
+  // units of this launch: part 0 every slot, 1 the routed experts' slots, 2 the shared
+  // expert's slot (one launch per bank when the banks' formats differ); every role walks
+  // u_begin + blockIdx.x, + gridDim.x, ... < total
+  const int u_begin = (part == 2) ? Ss.mt_prefix[n_active] * n_tiles : 0;
+  const int total = (part == 1) ? Ss.mt_prefix[n_active] * n_tiles : Ss.mt_prefix[n_slots] * n_tiles;
 
   auto fail = [&]() {
     set_status(p.status, DEV_TIMEOUT);
@@ -538,7 +542,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // (or to two lanes of one warp, which then take turns) holds one back by the other.
     if (lane == 0) {
       int it = 0, ui = 0;
-      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++ui) {
+      for (int u = u_begin + (int)blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++ui) {
         const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
         const int src = t.shared ? 1 : 0;
         const int wrow = t.e * N + t.ntile * kTcM;
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int k0 = GATE_UP ? 0 : 2 * iss, k1 = GATE_UP ? kTcBK / 16 : 2 * iss + 2;
     bool aborted = false;
     int it = 0, tile = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x, ++tile) {
+    for (int u = u_begin + (int)blockIdx.x; u < total; u += gridDim.x, ++tile) {
       const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
       const int n_mma = (t.nrows + 15) & ~15;
       const uint32_t idesc = umma_idesc_f16(n_mma);
@@ -658,7 +662,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     bool aborted = false;
     int it = 0, ia = 0, ui = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x, ++ui) {
+    for (int u = u_begin + (int)blockIdx.x; u < total; u += gridDim.x, ++ui) {
       const int sbuf = ui & 1;
       aborted = aborted || *abort_flag;
       if (threadIdx.x == 64) TCT(2, ui, 0);
@@ -742,7 +746,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ activation producer
     if (lane == 0) {
       int it = 0;
-      for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
+      for (int u = u_begin + (int)blockIdx.x; u < total && !*abort_flag; u += gridDim.x) {
         const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
         const int bx = box_index(t.nrows);
         const int src = t.shared ? 1 : 0;
@@ -772,7 +776,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31 (warps 10..13)
     const int row = quarter * 32 + lane;     // weight row in the tile
     int tile = 0;
-    for (int u = blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
+    for (int u = u_begin + (int)blockIdx.x; u < total && !*abort_flag; u += gridDim.x, ++tile) {
       const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
       const int b = tile % C::ACC_BUFS;
       if (!mbar_wait(&acc_full[b], (tile / C::ACC_BUFS) & 1)) {
@@ -880,7 +884,7 @@ TcSched tc_sched_view(void* base, int E) {
 }
 
 template <int FMT, bool GATE_UP, int ACC>
-static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t* xg,
+static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t* xg, int part,
                                  cudaStream_t st) {
   using C = TcCfg<FMT, GATE_UP, ACC>;
   const int K = GATE_UP ? p.d : p.f;
@@ -890,7 +894,8 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
   TcMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const Bank* banks[2] = {&p.routed, &p.shared};
-  const int nexp[2] = {p.E, p.has_shared ? 1 : 0};
+  // weight maps of the banks this launch reads (FMT is theirs)
+  const int nexp[2] = {part == 2 ? 0 : p.E, (p.has_shared && part != 1) ? 1 : 0};
   for (int b = 0; b < 2; ++b) {
     if (nexp[b] == 0) continue;
     for (int mi = 0; mi < C::NM; ++mi) {
@@ -949,17 +954,29 @@ static cudaError_t launch_tc_fmt(const Plan& p, const TcSched& S, const uint16_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, maps, p, S);
+  return cudaLaunchKernelEx(&cfg, kern, maps, p, S, part);
 }
 
 template <bool GATE_UP, int ACC>
+static cudaError_t launch_tc_part(const Plan& p, const TcSched& S, const uint16_t* xg, int fmt,
+                                  int part, cudaStream_t st) {
+  switch (fmt) {
+    case 4: return launch_tc_fmt<4, GATE_UP, ACC>(p, S, xg, part, st);
+    case 8: return launch_tc_fmt<8, GATE_UP, ACC>(p, S, xg, part, st);
+    default: return launch_tc_fmt<16, GATE_UP, ACC>(p, S, xg, part, st);
+  }
+}
+
+// One launch for both banks when they share a format; otherwise the routed experts and the
+// shared expert in two launches, each with its own format.
+template <bool GATE_UP, int ACC>
 static cudaError_t launch_tc(const Plan& p, const TcSched& S, const uint16_t* xg,
                              cudaStream_t st) {
-  switch (p.routed.fmt) {
-    case 4: return launch_tc_fmt<4, GATE_UP, ACC>(p, S, xg, st);
-    case 8: return launch_tc_fmt<8, GATE_UP, ACC>(p, S, xg, st);
-    default: return launch_tc_fmt<16, GATE_UP, ACC>(p, S, xg, st);
-  }
+  if (!p.has_shared || p.shared.fmt == p.routed.fmt)
+    return launch_tc_part<GATE_UP, ACC>(p, S, xg, p.routed.fmt, 0, st);
+  const cudaError_t err = launch_tc_part<GATE_UP, ACC>(p, S, xg, p.routed.fmt, 1, st);
+  if (err != cudaSuccess) return err;
+  return launch_tc_part<GATE_UP, ACC>(p, S, xg, p.shared.fmt, 2, st);
 }
 
 bool tc_supported(const Plan& p) {

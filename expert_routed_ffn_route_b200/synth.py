@@ -58,12 +58,13 @@ class LayerConfig:
     k: int          # routed experts per token
     f: int          # expert width (N of gate/up, K of down)
     n_shared: int = 1
-    fmt: str = "int4"            # routed and shared bank format
+    fmt: str = "int4"            # routed bank format (and the shared bank's by default)
     group: int = 128
     weight_std: float = 0.02
     zipf_s: float | None = None  # router bias popularity exponent (None: no bias)
     margin: float = 1e-3
     seed: int = 0
+    shared_fmt: str | None = None  # shared bank format when it differs from fmt
 
 
 # The five workloads. "tiny" is small enough for brute force on the CPU.
@@ -182,10 +183,11 @@ def make_bank(cfg: LayerConfig, which: str, n_exp: int | None = None,
     """
     if n_exp is None:
         n_exp = cfg.E if which == "routed" else cfg.n_shared
+    fmt = cfg.shared_fmt if (which == "shared" and cfg.shared_fmt) else cfg.fmt
     d, f, g = cfg.d, cfg.f, cfg.group
-    wg, sg = _alloc(cfg.fmt, n_exp, f, d, g)
-    wu, su = _alloc(cfg.fmt, n_exp, f, d, g)
-    wd, sd = _alloc(cfg.fmt, n_exp, d, f, g)
+    wg, sg = _alloc(fmt, n_exp, f, d, g)
+    wu, su = _alloc(fmt, n_exp, f, d, g)
+    wd, sd = _alloc(fmt, n_exp, d, f, g)
     todo = range(n_exp) if experts is None else experts
     jobs = [(int(e), name, shape, wa, sa) for e in todo
             for name, shape, wa, sa in (("gate", (f, d), wg, sg), ("up", (f, d), wu, su),
@@ -194,7 +196,7 @@ def make_bank(cfg: LayerConfig, which: str, n_exp: int | None = None,
     def one(job):
         e, name, shape, wa, sa = job
         w = _normal(shape, cfg.weight_std, cfg.seed, which, name, e)
-        q, s = _encode(w, cfg.fmt, g)
+        q, s = _encode(w, fmt, g)
         wa[e] = q
         if sa is not None:
             sa[e] = s
@@ -205,7 +207,7 @@ def make_bank(cfg: LayerConfig, which: str, n_exp: int | None = None,
     else:
         with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
             list(ex.map(one, jobs))
-    return Bank(cfg.fmt, g, n_exp, d, f, wg, wu, wd, sg, su, sd)
+    return Bank(fmt, g, n_exp, d, f, wg, wu, wd, sg, su, sd)
 
 
 def make_router(cfg: LayerConfig):

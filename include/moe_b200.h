@@ -36,6 +36,10 @@
  *       MOE_W_INT4  W[e][n][k / 8] uint32, 8 two's-complement nibbles per word along K,
  *                   element k at bits 4 * (k % 8) of word k / 8; scales as for int8.
  *     gate and up are [n_exp][f][d] (N = f, K = d); down is [n_exp][d][f] (N = d, K = f).
+ *     The two banks may use different encodings (e.g. an int8 shared expert beside int4
+ *     routed experts); the grouped products then run once per bank. The single-kernel
+ *     1-token path and the TMA GEMV path need int4 in both banks; other calls take the
+ *     register-streaming GEMV or the tensor-core path.
  *   - Supported shapes: 1 <= T, d % 128 == 0, f % 128 == 0, 1 <= k <= min(E, 32),
  *     1 <= E <= 1024, group == 128 for the integer formats, shared.n_exp in {0, 1}.
  */

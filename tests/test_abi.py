@@ -59,8 +59,10 @@ def test_validation_banks(lib):
     d.shared.n_exp = 2
     assert lib.moe_validate(ctypes.byref(d)) == -2
     d = _desc()
-    d.shared.fmt = 8
-    assert lib.moe_validate(ctypes.byref(d)) == -2
+    d.shared.fmt = 8  # an int8 shared expert beside int4 routed experts
+    assert lib.moe_validate(ctypes.byref(d)) == 0
+    d.shared.group = 64
+    assert lib.moe_validate(ctypes.byref(d)) == -1
     d = _desc()
     d.routed.s_up = None
     assert lib.moe_validate(ctypes.byref(d)) == -1

@@ -225,6 +225,18 @@ def test_tc_formats_many_rows_per_expert(B, fmt):
     check_layer(B, B.DeviceLayer(L), L, L.x, "tc")
 
 
+@pytest.mark.parametrize("routed,shared", [("int4", "int8"), ("int8", "int4"), ("int4", "bf16")])
+@pytest.mark.parametrize("T,path", [(1, "auto"), (5, "gemv"), (96, "tc")])
+def test_mixed_bank_formats(B, routed, shared, T, path):
+    """The shared expert in another encoding than the routed experts: the grouped products
+    run once per bank (the single-kernel and TMA GEMV paths decline such layers)."""
+    cfg = synth.LayerConfig(f"mixed-{routed}-{shared}", T=T, d=384, E=12, k=3, f=256,
+                            n_shared=1, fmt=routed, shared_fmt=shared, seed=19)
+    L = synth.make_layer(cfg)
+    assert L.shared.fmt == shared and L.routed.fmt == routed
+    check_layer(B, B.DeviceLayer(L), L, L.x, path)
+
+
 def test_tc_tiny(B, tiny):
     L, dl = tiny
     check_layer(B, dl, L, L.x, "tc")

@@ -41,3 +41,14 @@ def test_zipf_bias_skews_load():
     cnt = np.bincount(idx.ravel(), minlength=cfg.E)
     mean = idx.size / cfg.E
     assert cnt.max() > 10 * mean
+
+
+def test_shared_bank_format_option():
+    """shared_fmt draws the shared bank in its own encoding; the routed bank is unchanged."""
+    base = synth.LayerConfig("m", T=4, d=256, E=4, k=2, f=128, fmt="int4", seed=3)
+    mixed = synth.LayerConfig("m", T=4, d=256, E=4, k=2, f=128, fmt="int4", shared_fmt="int8",
+                              seed=3)
+    a, b = synth.make_layer(base), synth.make_layer(mixed)
+    assert b.shared.fmt == "int8" and b.routed.fmt == "int4"
+    assert np.array_equal(a.routed.w_gate, b.routed.w_gate)
+    assert b.shared.w_gate.dtype == np.int8 and np.abs(b.shared.w_gate.astype(np.int32)).max() <= 127
