@@ -86,13 +86,44 @@ KERNEL_SOURCES = {
 }
 
 
-def kernel_source_digest(kernel="gemv_tma"):
-    """Digest of the sources of one gate/up kernel (ties committed ncu counters to a build)."""
+def source_tokens(text):
+    """C/C++/CUDA source with comments removed and whitespace collapsed: what the compiler
+    sees, so that edits to comments alone keep a digest."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":  # string or character literal, kept whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
+def kernel_source_digest(kernel="gemv_tma", read=None):
+    """Digest of the sources of one kernel, comments and whitespace aside (ties committed ncu
+    counters to the code they were taken from). ``read`` maps a file name under csrc/ to its
+    text (default: the working tree)."""
     import hashlib
+    if read is None:
+        def read(name):
+            with open(os.path.join(ROOT, "expert_routed_ffn_route_b200", "csrc", name)) as fh:
+                return fh.read()
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "expert_routed_ffn_route_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        h.update(source_tokens(read(f)).encode())
     return h.hexdigest()[:16]
 
 

@@ -15,10 +15,11 @@
 //   warp 1      TMEM owner and MMA issuer (the whole warp, one elected lane issuing):
 //               tcgen05.mma kind::f16, fp32 accumulate; warp 14 issues in parallel into a
 //               separate accumulator (gate/up: the up projection; down: half the K steps)
-//   warps 2-9   dequantisers, two groups of four taking alternate chunks: W = fp16(q * s)
-//               written straight from registers into TMEM (tcgen05.st), where the MMA
-//               reads its A operand;
-//               shared memory then carries only the raw weights and the activations
+//   warps 2-9   dequantisers, two groups of four taking alternate steps of two 64-K chunks:
+//               W = fp16(q * s) written straight from registers into TMEM (tcgen05.st),
+//               where the MMA reads its A operand; each ready chunk is announced on a named
+//               barrier per A stage; shared memory carries only the raw weights and the
+//               activations
 //   warps 10-13 epilogue: tcgen05.ld of their 32 TMEM lanes; gate/up: h = silu(g) * u ->
 //               fp16 rows; down: fp32 rows
 //   warp 15     TMA producer of the activation tiles (warp 0 streams the weights)
