@@ -230,6 +230,29 @@ def test_shared_and_routed_parts_separate(tiny_layer):
     np.testing.assert_allclose(only_shared, h @ Wd.T, rtol=1e-10, atol=1e-14)
 
 
+
+def test_mixed_bank_formats_shared_part_is_dense_int8_swiglu():
+    """int4 routed experts beside an int8 shared expert: the layer minus its routed part is the
+    dense SwiGLU of the shared expert's dequantised int8 weights (q * s, group 128) on every
+    token, computed here with torch matmuls in fp64."""
+    cfg = synth.LayerConfig("mixed", T=7, d=256, E=6, k=2, f=128, n_shared=1, fmt="int4",
+                            shared_fmt="int8", seed=5)
+    L = synth.make_layer(cfg)
+    assert L.routed.fmt == "int4" and L.shared.fmt == "int8"
+    routed, shared = bank_dict(L.routed), bank_dict(L.shared)
+    full = O.layer_forward(L.x, L.router_w, L.router_bias, routed, shared, cfg.k)["out"]
+    no_shared = O.layer_forward(L.x, L.router_w, L.router_bias, routed, None, cfg.k)["out"]
+    X = torch.from_numpy(L.x.view(np.int16)).view(torch.bfloat16).to(torch.float64)
+    def W(q8, sb):
+        q = torch.from_numpy(q8.astype(np.float64))
+        s = torch.from_numpy(sb.view(np.int16)).view(torch.bfloat16).to(torch.float64)
+        return q * s.repeat_interleave(128, dim=1)
+    Wg, Wu, Wd = (W(getattr(L.shared, "w_" + n)[0], getattr(L.shared, "s_" + n)[0])
+                  for n in ("gate", "up", "down"))
+    F = torch.nn.functional
+    dense = F.linear(F.silu(F.linear(X, Wg)) * F.linear(X, Wu), Wd).numpy()
+    np.testing.assert_allclose(full - no_shared, dense, rtol=1e-9, atol=1e-13)
+
 # ------------------------------------------------------------ planted mistakes
 
 @pytest.mark.parametrize("mistake", ["tie_high_index", "silu_sign", "drop_shared",
