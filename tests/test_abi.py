@@ -89,3 +89,13 @@ def test_calls_reject_bad_arguments_before_any_cuda_call(lib):
                                  1 << 20, 1 << 40, None) == -1
     assert lib.moe_route(None, None, None, None, None, 0, None) == -1
     assert lib.moe_status_str(-4) == b"device-side wait timed out"
+
+
+@pytest.mark.parametrize("path,single", [(2, 5), (1, 4)])
+def test_launch_count_of_mixed_bank_formats(lib, path, single):
+    """16 tokens: routing (one launch), the grouped products, the combine; a shared bank in
+    another format than the routed one runs each of the two GEMMs once per bank."""
+    d = _desc(path=path)
+    assert lib.moe_launches_per_call(ctypes.byref(d)) == single
+    d.shared.fmt = 8
+    assert lib.moe_launches_per_call(ctypes.byref(d)) == single + 2
