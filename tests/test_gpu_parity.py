@@ -237,6 +237,28 @@ def test_mixed_bank_formats(B, routed, shared, T, path):
     check_layer(B, B.DeviceLayer(L), L, L.x, path)
 
 
+def test_gemv_path_row_invariance(B):
+    """On the GEMV path a token's output bits do not depend on the other tokens of the call
+    (up to 32): the first T rows of a 32-token call equal a T-token call bit for bit, and
+    permuting the tokens permutes the outputs bit for bit."""
+    cfg = synth.LayerConfig("ri", T=32, d=512, E=64, k=4, f=256, n_shared=1, fmt="int4", seed=23)
+    L = synth.make_layer(cfg)
+    dl = B.DeviceLayer(L)
+    x = torch.from_numpy(L.x.view(np.int16)).cuda().view(torch.bfloat16)
+
+    def run(xx):
+        desc = dl.descriptor(xx.shape[0], "gemv")
+        out = B.layer_forward(desc, xx.contiguous(), B.alloc_workspace(desc))
+        torch.cuda.synchronize()
+        return out.view(torch.int16)
+
+    o32 = run(x)
+    for T in (1, 2, 5, 16):
+        assert torch.equal(run(x[:T]), o32[:T]), T
+    perm = torch.randperm(32, generator=torch.Generator().manual_seed(1)).cuda()
+    assert torch.equal(run(x[perm]), o32[perm])
+
+
 def test_tc_tiny(B, tiny):
     L, dl = tiny
     check_layer(B, dl, L, L.x, "tc")
