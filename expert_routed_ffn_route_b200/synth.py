@@ -131,6 +131,62 @@ def quantize_groups(w: np.ndarray, qmax: int, group: int):
     return q.astype(np.int8).reshape(N, K), sb
 
 
+# ---------------------------------------------------------------- NVFP4 encoding
+# NVFP4 (NVIDIA's 4-bit floating-point weight format): E2M1 elements (magnitudes 0, 0.5, 1,
+# 1.5, 2, 3, 4, 6), one E4M3 scale per 16 consecutive elements along K, one float32 scale per
+# tensor; value = e2m1 * e4m3 * scale. Weights are encoded once here, in float32 arithmetic:
+# tensor scale g = amax / (6 * 448), block scale = E4M3(amax_block / (6 g)) (round to nearest
+# even, at most 448), element = E2M1(w / (block scale * g)) (round to nearest even, saturating
+# at 6). Codes: bit 3 sign, bits 2..1 exponent, bit 0 mantissa; two per byte, element k in the
+# nibble at bit 4 * (k % 2) of byte k // 2.
+NVFP4_BLOCK = 16
+_E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], np.float32)
+
+
+def e2m1_codes(v: np.ndarray) -> np.ndarray:
+    """float32 values -> E2M1 codes (uint8), nearest, ties to the even code, saturating."""
+    a = np.abs(v).astype(np.float32)
+    mids = (_E2M1_GRID[1:] + _E2M1_GRID[:-1]) / np.float32(2)
+    i = np.searchsorted(mids, a, side="left")  # mids strictly below a
+    tie = (i < len(mids)) & (a == mids[np.minimum(i, len(mids) - 1)])
+    i = np.where(tie & (i % 2 == 1), i + 1, i)
+    return (i.astype(np.uint8) | (np.signbit(v).astype(np.uint8) << 3)).astype(np.uint8)
+
+
+def e4m3_codes(v: np.ndarray) -> np.ndarray:
+    """Non-negative float32 values -> E4M3 (fn) codes, nearest even, at most 448."""
+    import torch
+    c = np.minimum(np.asarray(v, np.float32), np.float32(448.0))
+    return torch.from_numpy(np.ascontiguousarray(c)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def e4m3_to_f32(codes: np.ndarray) -> np.ndarray:
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float32).numpy()
+
+
+def quantize_nvfp4(w: np.ndarray):
+    """float32 [N, K] -> (packed codes uint8 [N, K/2], block scales uint8 [N, K/16],
+    tensor scale float32)."""
+    N, K = w.shape
+    assert K % NVFP4_BLOCK == 0
+    w = np.asarray(w, np.float32)
+    g = np.float32(np.abs(w).max() / np.float32(6.0 * 448.0))
+    wb = w.reshape(N, K // NVFP4_BLOCK, NVFP4_BLOCK)
+    if g == 0:
+        return (np.zeros((N, K // 2), np.uint8), np.zeros((N, K // NVFP4_BLOCK), np.uint8), g)
+    amax_b = np.abs(wb).max(axis=-1)
+    sc = e4m3_codes(amax_b / (np.float32(6.0) * g))
+    scale = (e4m3_to_f32(sc) * g).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0))
+    codes = e2m1_codes((wb / safe[..., None]).astype(np.float32))
+    codes[scale == 0] = 0
+    codes = codes.reshape(N, K)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed, sc, g
+
+
 @dataclass
 class Bank:
     """One expert bank: n_exp experts of gate [f,d], up [f,d], down [d,f]."""
@@ -145,10 +201,17 @@ class Bank:
     s_gate: np.ndarray | None = None
     s_up: np.ndarray | None = None
     s_down: np.ndarray | None = None
+    # nvfp4 only: one float32 scale per (expert, matrix)
+    g_gate: np.ndarray | None = None
+    g_up: np.ndarray | None = None
+    g_down: np.ndarray | None = None
 
     def arrays(self):
-        return dict(w_gate=self.w_gate, w_up=self.w_up, w_down=self.w_down,
-                    s_gate=self.s_gate, s_up=self.s_up, s_down=self.s_down)
+        a = dict(w_gate=self.w_gate, w_up=self.w_up, w_down=self.w_down,
+                 s_gate=self.s_gate, s_up=self.s_up, s_down=self.s_down)
+        if self.fmt == "nvfp4":
+            a.update(g_gate=self.g_gate, g_up=self.g_up, g_down=self.g_down)
+        return a
 
 
 def _encode(w: np.ndarray, fmt: str, group: int):
@@ -184,6 +247,8 @@ def make_bank(cfg: LayerConfig, which: str, n_exp: int | None = None,
     if n_exp is None:
         n_exp = cfg.E if which == "routed" else cfg.n_shared
     fmt = cfg.shared_fmt if (which == "shared" and cfg.shared_fmt) else cfg.fmt
+    if fmt == "nvfp4":
+        return _make_nvfp4_bank(cfg, which, n_exp, experts)
     d, f, g = cfg.d, cfg.f, cfg.group
     wg, sg = _alloc(fmt, n_exp, f, d, g)
     wu, su = _alloc(fmt, n_exp, f, d, g)
@@ -208,6 +273,25 @@ def make_bank(cfg: LayerConfig, which: str, n_exp: int | None = None,
         with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
             list(ex.map(one, jobs))
     return Bank(fmt, g, n_exp, d, f, wg, wu, wd, sg, su, sd)
+
+
+def _make_nvfp4_bank(cfg: LayerConfig, which: str, n_exp: int, experts=None) -> Bank:
+    """An NVFP4 bank over the same weight draws as the other formats."""
+    d, f = cfg.d, cfg.f
+    arrs = {}
+    for name, (N, K) in (("gate", (f, d)), ("up", (f, d)), ("down", (d, f))):
+        arrs[name] = (np.zeros((n_exp, N, K // 2), np.uint8),
+                      np.zeros((n_exp, N, K // NVFP4_BLOCK), np.uint8),
+                      np.zeros(n_exp, np.float32))
+    todo = range(n_exp) if experts is None else experts
+    for e in todo:
+        for name, (N, K) in (("gate", (f, d)), ("up", (f, d)), ("down", (d, f))):
+            w = _normal((N, K), cfg.weight_std, cfg.seed, which, name, int(e))
+            q, sc, g = quantize_nvfp4(w)
+            arrs[name][0][e], arrs[name][1][e], arrs[name][2][e] = q, sc, g
+    return Bank("nvfp4", NVFP4_BLOCK, n_exp, d, f, arrs["gate"][0], arrs["up"][0], arrs["down"][0],
+                arrs["gate"][1], arrs["up"][1], arrs["down"][1],
+                arrs["gate"][2], arrs["up"][2], arrs["down"][2])
 
 
 def make_router(cfg: LayerConfig):
