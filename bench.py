@@ -3,15 +3,20 @@
 
 A step is one full layer call (route -> plan -> grouped gate/up + SwiGLU -> grouped
 down -> combine) over one batch of synthetic hidden states, on weights resident in
-HBM. Default workload: 1-token decode (d=2560, E=512, top-10 + 1 shared, f=1024,
-int4 g128). Prints ONE JSON line on rank 0.
+HBM. The default run measures the five workloads of the metric (MoE-layer tokens/s at
+T = 1, 16, 32, 512, 4096) in one process and prints ONE JSON line on rank 0: the 1-token
+decode workload (d=2560, E=512, top-10 + 1 shared, f=1024, int4 g128) is the headline
+``value``; every workload has its entry in ``workloads``.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|NAME]
     python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
 
-L2: each step reads a different copy of the layer's weights (``replicas`` copies,
-cycled) and a different hidden batch (a pool of 64), so no step finds its weights in
-the 126 MB L2 (the inputs of the cycle are far larger than L2).
+Timing: the K steps of a workload are captured into CUDA graphs; the K-step region is
+replayed until at least ``--min-seconds`` have passed, each replay timed with CUDA events
+on the launch stream, and the median per-step time over the replays is reported.
+L2: each step reads a different copy of the layer's weights (``replicas`` copies, cycled)
+and a different hidden batch (a pool of 64), so no step finds its weights in the 126 MB L2
+(the inputs of the cycle are far larger than L2).
 Multi-GPU: every rank runs its own replica of the layer (weak scaling, no data-path
 collective); the time is the max over ranks.
 """
@@ -32,32 +37,39 @@ sys.path.insert(0, ROOT)
 from expert_routed_ffn_route_b200 import synth  # noqa: E402
 
 HBM_FALLBACK_GBS = 6650.0
+TC_FALLBACK_TFLOPS = 1590.0
+HBM_NOMINAL_GBS = 8000.0      # the HBM3e figure the decode target is stated against
+TC_NOMINAL_TFLOPS = 2250.0    # dense bf16/fp16 tensor-core peak of one B200
 L2_BYTES = 126 * 2 ** 20
 POOL = 64
+ALL_WORKLOADS = ("decode", "verify16", "verify32", "prefill", "long")
+HEADLINE = "decode"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=list(synth.CONFIGS))
+    ap.add_argument("--workload", default="all", choices=["all", *synth.CONFIGS])
     ap.add_argument("--replicas", type=int, default=0, help="weight copies cycled (0: auto)")
-    ap.add_argument("--no-graph", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--stage-times", action="store_true",
-                    help="also report per-stage CUDA-event times (stage marks block overlap)")
-    return ap.parse_args()
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="replay the K-step region until this much time has passed")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return ap.parse_args(argv)
 
 
 def measured_peaks():
+    """(hbm GB/s, tensor TFLOP/s burst, tensor TFLOP/s sustained, kind)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as fh:
             d = json.load(fh)
-        return float(d["hbm_gbs"]), "measured"
-    return HBM_FALLBACK_GBS, "fallback"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
+    return HBM_FALLBACK_GBS, TC_FALLBACK_TFLOPS, TC_FALLBACK_TFLOPS, "fallback"
 
 
 def bank_bytes_per_expert(cfg):
@@ -65,6 +77,42 @@ def bank_bytes_per_expert(cfg):
     w = 3 * cfg.d * cfg.f * bits // 8
     s = 0 if cfg.fmt == "bf16" else 3 * cfg.d * cfg.f // cfg.group * 2
     return w, s
+
+
+def layer_flops(cfg):
+    """Algorithmic FLOPs of one layer call: 2 * 3 * d * f per (token, expert) pair, over
+    the T * k routed pairs and the T shared-expert rows (the router's 2 * T * E * d is
+    included too)."""
+    return (2 * 3 * cfg.d * cfg.f * (cfg.T * cfg.k + cfg.T * cfg.n_shared)
+            + 2 * cfg.T * cfg.E * cfg.d)
+
+
+def pool_size(cfg):
+    """Hidden batches cycled: 64 for the small calls (each touches few experts, so the
+    batches must differ), fewer for large T (every batch touches nearly every expert)."""
+    return int(min(POOL, max(4, 4096 // cfg.T)))
+
+
+def replicas_for(cfg, requested=0):
+    """Weight copies cycled: enough that a cycle of steps touches more than 4x L2."""
+    if requested > 0:
+        return requested
+    w_b, s_b = bank_bytes_per_expert(cfg)
+    touched = min(cfg.E, cfg.T * cfg.k) + 1
+    step_bytes = touched * (w_b + s_b) + cfg.E * cfg.d * 2
+    return int(min(16, max(1, np.ceil(4 * L2_BYTES / step_bytes))))
+
+
+def workload_config(cfg, world, replicas=0):
+    """The ``config`` object of a bench line (identical for both arms)."""
+    R = replicas_for(cfg, replicas)
+    return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+            "f": cfg.f, "n_shared": cfg.n_shared, "weights": f"{cfg.fmt} g{cfg.group}",
+            "router": "bf16, fp32 logits" + (", Zipf(1.1) bias" if cfg.zipf_s else ""),
+            "parallelism": f"replicas x{world}",
+            "l2": (f"inputs larger than L2: {R} weight copies x {pool_size(cfg)} hidden "
+                   "batches cycled"),
+            "cuda_graph": True}
 
 
 def max_over_ranks(values, device="cpu"):
@@ -127,7 +175,7 @@ def kernel_source_digest(kernel="gemv_tma", read=None):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload, kernel="gemv_tma"):
+def profiled_traffic(workload, kernel):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary
     ``profiles/<kernel>_gate_up_<workload>.md`` (``profiles/<kernel>_<workload>.md`` for the
     single-kernel layer), if it was captured from the current kernel sources (else None)."""
@@ -146,49 +194,81 @@ def profiled_traffic(workload, kernel="gemv_tma"):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_rate(cfg, L, seconds):
-    """Tokens/s of the fp64 oracle on this host, on a bounded sample of the workload:
-    whole calls of up to 1 token each on successive tokens until `seconds` pass."""
-    from oracle import moe_oracle as O
+def _oracle_bank(b):
+    if b is None:
+        return None
+    d = b.arrays()
+    d.update(fmt=b.fmt, group=b.group)
+    return d
 
-    def bank_dict(b):
-        if b is None:
-            return None
-        d = b.arrays()
-        d.update(fmt=b.fmt, group=b.group)
-        return d
-    routed, shared = bank_dict(L.routed), bank_dict(L.shared)
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+# Tokens of the batched oracle call timed per workload: the whole batch where that ends in
+# seconds, else the first tokens of it (the oracle dequantises each touched expert once per
+# call, about 0.1 s an expert, so its cost grows with the experts a slice touches).
+CPU_SLICE = {"tiny": 64, "decode": 1, "verify16": 8, "verify32": 8, "prefill": 16, "long": 64}
+
+
+def cpu_oracle_rate(cfg, L, seconds, n_tokens=None):
+    """Tokens/s of the fp64 oracle on this host, on a bounded sample of the workload: batched
+    layer calls on the first ``n_tokens`` tokens of the batch (every touched expert
+    dequantised once per call, as the workload's own call does), repeated until ``seconds``
+    pass (at least one call)."""
+    from oracle import moe_oracle as O
+    routed, shared = _oracle_bank(L.routed), _oracle_bank(L.shared)
+    n = L.x.shape[0] if n_tokens is None else min(n_tokens, L.x.shape[0])
+    x = L.x[:n]
     t0 = time.perf_counter()
-    done = 0
+    done = calls = 0
     while True:
-        t = done % L.x.shape[0]
-        O.layer_forward(L.x[t:t + 1], L.router_w, L.router_bias, routed, shared, cfg.k)
-        done += 1
+        O.layer_forward(x, L.router_w, L.router_bias, routed, shared, cfg.k)
+        done += n
+        calls += 1
         if time.perf_counter() - t0 >= seconds:
             break
     el = time.perf_counter() - t0
-    cores = os.cpu_count()
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        pass
-    return done / el, cores, f"{done} single-token layer calls of '{cfg.name}' in {el:.1f} s"
+    sample = (f"{calls} batched layer call(s) on the first {n} of the {cfg.T} tokens of "
+              f"'{cfg.name}' (each touched expert dequantised once a call) in {el:.1f} s")
+    return done / el, _blas_threads(), sample
 
 
-def cpu_baseline(cfg, L, seconds):
-    """The oracle's tokens/s with the host's BLAS threads (``value``) and with one thread
-    (``value_1thread``, on a sample of a third of the time)."""
-    rate, cores, sample = cpu_oracle_rate(cfg, L, seconds)
+def cpu_baseline(cfg, L, seconds, one_thread=True):
+    """The oracle's tokens/s with the host's BLAS threads (``value``) and, for the headline,
+    with one thread (``value_1thread``)."""
+    n = CPU_SLICE.get(cfg.name)
+    rate, cores, sample = cpu_oracle_rate(cfg, L, seconds, n)
     out = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+    if not one_thread:
+        return out
     try:
         from threadpoolctl import threadpool_limits
     except Exception:
         return out
     with threadpool_limits(limits=1):
-        r1, _, s1 = cpu_oracle_rate(cfg, L, seconds / 3)
+        r1, _, s1 = cpu_oracle_rate(cfg, L, seconds / 3, n)
     out.update(value_1thread=r1, sample_1thread=s1)
     return out
+
+
+def oracle_inputs(cfg, n_tokens=None):
+    """Inputs of a workload for the oracle with only the experts its tokens touch drawn
+    (the others are never read); ``n_tokens`` restricts the call to its first tokens."""
+    from oracle import moe_oracle as O
+    L = synth.make_layer(cfg, routed=synth.make_bank(cfg, "routed", experts=[]),
+                         shared=synth.make_bank(cfg, "shared") if cfg.n_shared else None)
+    n_tokens = CPU_SLICE.get(cfg.name) if n_tokens is None else n_tokens
+    if n_tokens is not None:
+        L.x = L.x[:n_tokens]
+    need = np.unique(O.select_topk(O.router_logits(L.x, L.router_w, L.router_bias), cfg.k)[0])
+    L.routed = synth.make_bank(cfg, "routed", experts=need)
+    return L
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -244,38 +324,47 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def run_ours(args, rank, world, local_rank):
+class BankCache:
+    """Host-side weight banks, drawn once per (format, seed, shape) and reused by the
+    workloads that share them (decode, verify and prefill use one int4 bank)."""
+
+    def __init__(self):
+        self.banks = {}
+
+    def get(self, cfg, which):
+        key = (which, cfg.fmt if which == "routed" else (cfg.shared_fmt or cfg.fmt), cfg.seed,
+               cfg.d, cfg.f, cfg.E if which == "routed" else cfg.n_shared)
+        if key not in self.banks:
+            self.banks[key] = synth.make_bank(cfg, which)
+        return self.banks[key]
+
+
+def run_workload(name, args, world, local_rank, cache):
+    """Times one workload; returns its bench entry (and the host inputs)."""
     import torch
     from expert_routed_ffn_route_b200 import binding as B
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = synth.CONFIGS[args.workload]
-    B.load_library()
+    cfg = synth.CONFIGS[name]
 
     # ---- inputs
-    routed = synth.make_bank(cfg, "routed")
-    shared = synth.make_bank(cfg, "shared")
+    routed = cache.get(cfg, "routed")
+    shared = cache.get(cfg, "shared") if cfg.n_shared else None
     L = synth.make_layer(cfg, routed=routed, shared=shared)
+    n_pool = pool_size(cfg)
     pool = [L.x] + [synth.make_hidden(cfg, L.router_w, L.router_bias, stream=f"pool{i}")
-                    for i in range(1, POOL)]
+                    for i in range(1, n_pool)]
     base = B.DeviceLayer(L, device=dev)
     x_dev = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in pool]
 
     w_b, s_b = bank_bytes_per_expert(cfg)
     per_exp = w_b + s_b
     router_b = cfg.E * cfg.d * 2
-    # replicas: enough weight copies that a cycle touches > 4x L2
-    if args.replicas > 0:
-        R = args.replicas
-    else:
-        touched = min(cfg.E, cfg.T * cfg.k) + 1
-        step_bytes = touched * per_exp + router_b
-        R = int(min(16, max(1, np.ceil(4 * L2_BYTES / step_bytes))))
+    R = replicas_for(cfg, args.replicas)
     layers = [base]
     for _ in range(R - 1):
         b2 = {}
-        for name, bank in base.banks.items():
-            b2[name] = None if bank is None else {
+        for bn, bank in base.banks.items():
+            b2[bn] = None if bank is None else {
                 k: (v.clone() if hasattr(v, "clone") else v) for k, v in bank.items()}
         layers.append(B.DeviceLayer.from_tensors(
             cfg, base.router_w.clone(),
@@ -286,7 +375,7 @@ def run_ours(args, rank, world, local_rank):
     out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
     idx_buf = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
 
-    # ---- algorithmic bytes of the dominant kernel (grouped gate/up) per pool entry
+    # ---- algorithmic bytes per pool entry: the layer, and its grouped gate/up launch
     gu_bytes, layer_bytes = [], []
     for xd in x_dev:
         B.layer_forward(descs[0], xd, ws, out=out, topk_idx=idx_buf)
@@ -297,116 +386,106 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
-    n_mark = min(args.steps, 256)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(n_mark)]
-    for a, b in ev:  # torch creates the CUDA event on its first record
-        a.record(stream)
-        b.record(stream)
-
-    # The dominant kernel: the single-kernel layer when a call is one launch (its marks
-    # bracket the whole call), else the grouped gate/up kernel (marks 2 and 3).
     fused = B.launches_per_call(descs[0]) == 1
-    mark_pair = (0, B.N_MARKS - 1) if fused else (2, 3)
-    dom_bytes = layer_bytes if fused else gu_bytes
+    K = args.steps
 
-    def step(i, marked=False):
-        marks = None
-        if marked:
-            marks = [None] * B.N_MARKS
-            marks[mark_pair[0]], marks[mark_pair[1]] = ev[i % n_mark]
-        B.layer_forward(descs[i % R], x_dev[i % POOL], ws, out=out, marks=marks, stream=stream)
+    def step(i, marks=None):
+        B.layer_forward(descs[i % R], x_dev[i % n_pool], ws, out=out, marks=marks, stream=stream)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             step(i)
     torch.cuda.synchronize()
 
-    # The K timed steps are captured once into CUDA graphs of up to G steps each (a
-    # decode step is a few microseconds of GPU work; per-step host launches would
-    # dominate). A second, shorter pass with stage marks around the gate/up kernel gives
-    # that kernel's launch duration from CUDA events.
+    # K steps captured once into CUDA graphs of up to G steps each (a decode step is a few
+    # microseconds of GPU work; per-step host launches would dominate)
     G = 64
-    plain, marked = [], []
-    if not args.no_graph:
-        for a0 in range(0, args.steps, G):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for i in range(a0, min(args.steps, a0 + G)):
-                    step(i)
-            plain.append(g)
+    plain = []
+    for a0 in range(0, K, G):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(a0, min(K, a0 + G)):
+                step(i)
+        plain.append(g)
+    # the grouped gate/up launch of the multi-kernel path, bracketed by stage marks (CUDA
+    # events recorded on the launch stream; marks 2 and 3 enclose the gate/up stage)
+    n_mark = min(K, 256)
+    ev = []
+    marked = []
+    if not fused:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_mark)]
+        for a, b in ev:  # torch creates the CUDA event on its first record
+            a.record(stream)
+            b.record(stream)
         for a0 in range(0, n_mark, G):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for i in range(a0, min(n_mark, a0 + G)):
-                    step(i, marked=True)
+                    marks = [None] * B.N_MARKS
+                    marks[2], marks[3] = ev[i]
+                    step(i, marks)
             marked.append(g)
-        with torch.cuda.stream(stream):  # one untimed pass over every graph
-            for g in plain + marked:
-                g.replay()
-        torch.cuda.synchronize()
+    with torch.cuda.stream(stream):  # one untimed pass over every graph
+        for g in plain + marked:
+            g.replay()
+    torch.cuda.synchronize()
 
-    def run(graphs, n, with_marks):
+    def replay(graphs):
         with torch.cuda.stream(stream):
-            if graphs:
-                for g in graphs:
-                    g.replay()
-            else:
-                for i in range(n):
-                    step(i, marked=with_marks)
+            for g in graphs:
+                g.replay()
 
-    # ---- timed region
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    # ---- timed regions: the K-step region replayed until min_seconds have passed
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
+    region_ms = []
     with ClockSampler(local_rank) as clk:
-        time.sleep(0.3)  # let the sampler start before the timed region
-        torch.cuda.nvtx.range_push("timed")
-        t_start.record(stream)
-        run(plain, args.steps, False)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-        torch.cuda.nvtx.range_pop()
+        time.sleep(0.25)  # let the sampler start before the timed regions
+        t_wall = time.perf_counter()
+        while True:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            replay(plain)
+            e1.record(stream)
+            e1.synchronize()
+            region_ms.append(e0.elapsed_time(e1))
+            if time.perf_counter() - t_wall >= args.min_seconds and len(region_ms) >= 3:
+                break
     if world > 1:
         dist.barrier()
-    ms = t_start.elapsed_time(t_end)
+    ms_region = float(np.median(region_ms))
+    (ms_region,) = max_over_ranks([ms_region], device=dev)
+    ms_per_step = ms_region / K
 
-    # dominant kernel: gate/up launches of the marked pass (CUDA events on the launch stream)
-    torch.cuda.synchronize()
-    run(marked, n_mark, True)
-    torch.cuda.synchronize()
-    k_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n_mark)]
-    k_bytes = [dom_bytes[i % POOL] for i in range(n_mark)]
-    gu_avg_ms = float(np.mean(k_ms))
-    achieved = float(np.sum(k_bytes) / (np.sum(k_ms) * 1e-3) / 1e9)
-
-    stage_ms = None
-    if args.stage_times:
-        n_st = min(args.steps, 200)
-        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(B.N_MARKS)]
-               for _ in range(n_st)]
-        for row in sev:  # torch creates the CUDA event on its first record
-            for e_ in row:
-                e_.record(stream)
-        with torch.cuda.stream(stream):
-            for i in range(n_st):
-                B.layer_forward(descs[i % R], x_dev[i % POOL], ws, out=out, marks=sev[i],
-                                stream=stream)
+    # ---- dominant kernel: the single-kernel layer is the whole step; otherwise the gate/up
+    # launch from the marked pass
+    if fused:
+        k_ms_avg = ms_per_step
+        achieved = float(np.mean([layer_bytes[i % n_pool] for i in range(K)])) / (ms_per_step * 1e-3) / 1e9
+        kernel_name = "decode_fused_kernel (whole layer, one launch)"
+        prof_kernel = "decode_fused"
+    else:
         torch.cuda.synchronize()
-        names = ["route", "plan", "gate_up", "down", "combine"]
-        stage_ms = {n: float(np.mean([sev[i][j].elapsed_time(sev[i][j + 1])
-                                      for i in range(n_st // 2, n_st)]))
-                    for j, n in enumerate(names)}
+        replay(marked)
+        torch.cuda.synchronize()
+        k_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n_mark)]
+        k_bytes = [gu_bytes[i % n_pool] for i in range(n_mark)]
+        k_ms_avg = float(np.mean(k_ms))
+        achieved = float(np.sum(k_bytes) / (np.sum(k_ms) * 1e-3) / 1e9)
+        tc = cfg.T >= 16
+        kernel_name = "grouped gate/up + SwiGLU" + (" (tcgen05, with its row gather)" if tc else "")
+        prof_kernel = "tc_grouped" if tc else "gemv_tma"
 
     # ---- end to end through the public call with host buffers
     x_host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
               for x in pool[:8]]
     out_host = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16).pin_memory()
     x_stage = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
-    e_steps = min(args.steps, 200)
+    e_steps = max(8, min(K, 200))
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -419,89 +498,128 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e_steps
+    (e2e_ms,) = max_over_ranks([e2e_ms], device=dev)
     status = B.device_status(descs[0], ws)
 
-    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
-
-    peak, peak_kind = measured_peaks()
-    ms_per_step = ms / args.steps
-    res = {
+    hbm, tc_burst, tc_sust, peak_kind = measured_peaks()
+    lb = float(np.mean(layer_bytes))
+    layer_gbs = lb / (ms_per_step * 1e-3) / 1e9
+    flops = layer_flops(cfg)
+    tflops = flops / (ms_per_step * 1e-3) / 1e12
+    roof = {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": hbm,
+            "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
+            "frac_nominal": achieved / HBM_NOMINAL_GBS,
+            "traffic": profiled_traffic(cfg.name, prof_kernel),
+            "avg_launch_ms": k_ms_avg,
+            "layer_bytes": lb, "layer_achieved": layer_gbs, "layer_frac": layer_gbs / hbm,
+            "layer_frac_nominal": layer_gbs / HBM_NOMINAL_GBS,
+            "tensor": {"flops_per_step": flops, "achieved_tflops": tflops,
+                       "peak_sustained": tc_sust, "frac": tflops / tc_sust,
+                       "peak_burst": tc_burst, "frac_burst": tflops / tc_burst,
+                       "peak_nominal": TC_NOMINAL_TFLOPS,
+                       "frac_nominal": tflops / TC_NOMINAL_TFLOPS}}
+    entry = {
         "metric": f"MoE-layer tokens/s ({cfg.name}, T={cfg.T})",
-        "value": world * cfg.T * args.steps / (ms * 1e-3),
+        "value": world * cfg.T / (ms_per_step * 1e-3),
         "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": ms_per_step,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
+        "steps": K,
+        "regions": len(region_ms),
+        "region_ms": {"median": ms_region, "min": float(np.min(region_ms)),
+                      "max": float(np.max(region_ms))},
         "dtype": f"{cfg.fmt} weights, bf16 activations, fp32 accumulate",
-        "data": "synthetic (seeded; shapes of the pages' model, random weights)",
-        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "f": cfg.f, "n_shared": cfg.n_shared, "weights": f"{cfg.fmt} g{cfg.group}",
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: {R} weight copies x {POOL} hidden batches cycled",
-                   "cuda_graph": not args.no_graph},
-        "roofline": {"bound": "hbm",
-                     "kernel": ("decode_fused_kernel (whole layer, one launch)" if fused
-                                else "grouped gate/up + SwiGLU"),
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": profiled_traffic(cfg.name, "decode_fused" if fused else
-                                                 ("tc_grouped" if cfg.T >= 16 else "gemv_tma")),
-                     "avg_launch_ms": gu_avg_ms,
-                     "layer_frac": float(np.mean(layer_bytes)) / (ms_per_step * 1e-3) / 1e9 / peak},
+        "config": workload_config(cfg, world, args.replicas),
+        "roofline": roof,
         "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
-        "gpu_launches": B.launches_per_call(descs[0]) * args.steps,
+        "gpu_launches_per_step": B.launches_per_call(descs[0]),
         "clocks": clk.summary(),
         "device_status": status,
-        **({"stages_ms_eager": stage_ms} if stage_ms else {}),
     }
-    return res, L, cfg
+    if cfg.T >= 512:  # the tensor-core workloads: the contraction's share of the roofline
+        roof["tc_frac"] = roof["tensor"]["frac"]
+    del layers, base, descs, ws, x_dev
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry, L, cfg
 
 
-def main():
-    args = parse()
+def main(argv=None):
+    args = parse(argv)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
-    cfg = synth.CONFIGS[args.workload]
+    names = list(ALL_WORKLOADS) if args.workload == "all" else [args.workload]
+    head = HEADLINE if args.workload == "all" else args.workload
 
     if args.impl == "reference":
         if rank != 0:
             return 0
-        L = synth.make_layer(cfg, routed=synth.make_bank(cfg, "routed", experts=[]),
-                             shared=synth.make_bank(cfg, "shared"))
-        # only the experts the sampled tokens touch are drawn (others are never read)
-        from oracle import moe_oracle as O
-        need = np.unique(O.select_topk(O.router_logits(L.x[:64], L.router_w, L.router_bias),
-                                       cfg.k)[0])
-        L.routed = synth.make_bank(cfg, "routed", experts=need)
-        cb = cpu_baseline(cfg, L, args.cpu_seconds)
+        cfg = synth.CONFIGS[head]
+        L = oracle_inputs(cfg)
+        t0 = time.perf_counter()
+        cb = cpu_baseline(cfg, L, args.cpu_seconds, one_thread=False)
         rate = cb["value"]
         line = {"impl": "reference", "metric": f"MoE-layer tokens/s ({cfg.name}, T={cfg.T})",
-                "value": rate, "unit": "tokens/s", "n_gpus": 0, "steps": args.steps,
-                "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "value": rate, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * cfg.T / rate,
+                "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": cfg.name, "T": cfg.T},
+                "config": workload_config(cfg, world, args.replicas),
                 "cpu_baseline": cb,
                 "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
+                        "d2h_bytes_per_step": 0},
+                "wall_s": time.perf_counter() - t0}
         print(json.dumps(line))
         return 0
 
+    import torch
+    torch.cuda.set_device(local_rank)
     if world > 1:
-        import torch
         import torch.distributed as dist
         from datetime import timedelta
-        torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    res, L, cfg = run_ours(args, rank, world, local_rank)
-    if rank == 0 and world == 1:
-        res["cpu_baseline"] = cpu_baseline(cfg, L, args.cpu_seconds)
+    from expert_routed_ffn_route_b200 import binding as B
+    B.load_library()
+    cache = BankCache()
+    entries, inputs = {}, {}
+    for n in names:
+        entries[n], L, cfg = run_workload(n, args, world, local_rank, cache)
+        inputs[n] = (L, cfg)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        for n in names:
+            L, cfg = inputs[n]
+            entries[n]["cpu_baseline"] = cpu_baseline(cfg, L, args.cpu_seconds,
+                                                      one_thread=(n == head))
+    cache.banks.clear()
+    h = entries[head]
+    res = {
+        "metric": h["metric"],
+        "value": h["value"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": h["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": h["dtype"],
+        "data": "synthetic (seeded; shapes of the pages' model, random weights)",
+        "config": h["config"],
+        "roofline": h["roofline"],
+        "e2e": h["e2e"],
+        "gpu_launches": h["gpu_launches_per_step"] * args.steps,
+        "clocks": h["clocks"],
+        "device_status": h["device_status"],
+        "timing": (f"median over {h['regions']} replays of the {args.steps}-step region "
+                   f"(each >= {args.min_seconds} s in total), CUDA events on the launch stream"),
+    }
+    if "cpu_baseline" in h:
+        res["cpu_baseline"] = h["cpu_baseline"]
+    if len(names) > 1:
+        res["workloads"] = entries
     if rank == 0:
         print(json.dumps(res))
     if world > 1:

@@ -46,7 +46,7 @@ _LIB = None
 EXPORTS = ["moe_abi_version", "moe_status_str", "moe_validate", "moe_workspace_size",
            "moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
            "moe_layer_forward_marked", "moe_device_status", "moe_launches_per_call",
-           "moe_layer_forward_static"]
+           "moe_layer_forward_static", "moe_static_device_status", "moe_test_inject_hold"]
 
 
 def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
@@ -78,6 +78,8 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "moe_device_status": (I32, [LP, P, SZ, ctypes.POINTER(I32), P]),
         "moe_launches_per_call": (I32, [LP]),
         "moe_layer_forward_static": (I32, [LP, P, P, P]),
+        "moe_static_device_status": (I32, [ctypes.POINTER(I32), P]),
+        "moe_test_inject_hold": (I32, [LP, P, SZ, I32, I32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -262,3 +264,18 @@ def layer_forward_static(L: MoeLayer, x, out=None, stream=None):
                                                    out.data_ptr(), _stream(stream)),
            "moe_layer_forward_static")
     return out
+
+
+def static_device_status(stream=None) -> int:
+    """Reads and clears the status word of the built-in scratch (moe_layer_forward_static)."""
+    code = ctypes.c_int32(0)
+    _check(load_library().moe_static_device_status(ctypes.byref(code), _stream(stream)),
+           "moe_static_device_status")
+    return code.value
+
+
+def test_inject_hold(L: MoeLayer, ws, hold: bool, budget_cycles: int = 0, stream=None):
+    """Sets or clears the workspace's failure-injection hold word (see the header)."""
+    _check(load_library().moe_test_inject_hold(ctypes.byref(L), ws.data_ptr(), ws.numel(),
+                                               int(bool(hold)), int(budget_cycles),
+                                               _stream(stream)), "moe_test_inject_hold")

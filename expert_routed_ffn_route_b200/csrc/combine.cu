@@ -20,9 +20,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const float* __re
                                                                int d, int k) {
   __shared__ int s_row[kMaxK];
   __shared__ float s_w[kMaxK];
-  KT_ENTRY(4);
   pdl_wait();
-  KT_READY(4);
   const int t = blockIdx.y;
   if (threadIdx.x < k) {
     s_row[threadIdx.x] = inv[(size_t)t * k + threadIdx.x];
@@ -59,7 +57,6 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const float* __re
   o.x = pack_bf16x2(acc.x, acc.y);
   o.y = pack_bf16x2(acc.z, acc.w);
   *reinterpret_cast<uint2*>(out + (size_t)t * d + n) = o;
-  KT_EXIT(4);
 }
 
 cudaError_t launch_combine(const Plan& p, void* out, cudaStream_t st, bool pdl) {

@@ -49,19 +49,6 @@ constexpr int kDfMaxTiles = 8;
 constexpr int kDfMaxUnits = 24;
 constexpr int kDfMaxRouter = 8;
 
-#ifdef MOE_TRACE
-__device__ long long g_dftrace[160][32];
-#define DFT(slot) \
-  do { if (threadIdx.x == 0 && blockIdx.x < 160) { unsigned long long _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_dftrace[blockIdx.x][(slot)] = (long long)_t; } } while (0)
-extern "C" __attribute__((visibility("default"))) int moe_dftrace_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_dftrace, sizeof(g_dftrace));
-}
-#define DFTP(slot) \
-  do { if (blockIdx.x < 160) { unsigned long long _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_dftrace[blockIdx.x][(slot)] = (long long)_t; } } while (0)
-#else
-#define DFT(slot) do {} while (0)
-#define DFTP(slot) do {} while (0)
-#endif
 
 // Smem scratch beyond the buffers: picks, gates and the CTA's tile/unit tables.
 struct DfMisc {
@@ -150,37 +137,6 @@ __host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int
   o += (uint32_t)((sizeof(DfMisc) + 15) & ~size_t(15));
   L.total = o;
   return L;
-}
-
-// ------------------------------------------------------------------ grid barrier
-
-// Grid-wide barrier on one 32-bit word whose low 31 bits are zero between barriers (the
-// workspace starts zeroed). Every CTA adds to the word once per barrier; CTA 0 adds
-// 2^31 - (grid - 1) and the others 1, so the top bit flips exactly when the last CTA
-// arrives and the low bits are zero again afterwards. A CTA is through once it sees the
-// top bit differ from the value it found on arrival.
-__device__ __forceinline__ void fence_acq_rel_gpu() {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
-
-// Arrival: a release (this CTA's writes, ordered before it by the CTA barrier the caller
-// has passed, become visible to every CTA that sees the arrival).
-__device__ __forceinline__ uint32_t gbar_arrive(uint32_t* bar) {
-  const uint32_t add = (blockIdx.x == 0) ? (0x80000000u - (gridDim.x - 1)) : 1u;
-  fence_acq_rel_gpu();
-  return atomicAdd(bar, add);
-}
-
-__device__ __forceinline__ bool gbar_wait(const uint32_t* bar, uint32_t arrived) {
-  const long long t0 = clock64();
-  while (true) {
-    uint32_t now;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(bar) : "memory");
-    if ((now ^ arrived) & 0x80000000u) break;
-    if (clock64() - t0 > kWaitCycles) return false;
-    __nanosleep(32);
-  }
-  return true;
 }
 
 // A wait that every lane of the warp leaves with the same verdict.
@@ -278,10 +234,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
   const int c = blockIdx.x, grid = gridDim.x;
   const int r0 = (int)((long long)E * c / grid), r1 = (int)((long long)E * (c + 1) / grid);
   const int nr = r1 - r0;
-  DFT(0);
-#ifdef MOE_TRACE
-  if (tid == 0 && blockIdx.x < 160) g_dftrace[blockIdx.x][26] = clock64();
-#endif
 
   // ---------------------------------------------------------------- prologue
   const int t0 = (int)((long long)L.tiles_total * c / grid);
@@ -297,7 +249,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       for (int i = 0; i < kDfMaxTiles; ++i) mbar_init(&bar_tile[i], 1);
       for (int i = 0; i < kDfMaxUnits; ++i) mbar_init(&bar_unit[i], 1);
       fence_barrier_init();
-      DFTP(1);
       mi->ok = 1;
       mi->armed_tiles = has_sh_tile ? 1 : 0;
       mi->armed_units = 0;
@@ -316,14 +267,12 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         bulk_g2s(smem + 2 * wbytes, p.shared.s[0] + row * G, sbytes, &bar_tile[0]);
         bulk_g2s(smem + 2 * wbytes + sbytes, p.shared.s[1] + row * G, sbytes, &bar_tile[0]);
       }
-      DFTP(2);
     }
     __syncwarp();
   } else {
     // the activation row (bf16)
     for (int i = tid; i < d / 8; i += kDfCompute)
       reinterpret_cast<uint4*>(s_x)[i] = __ldg(reinterpret_cast<const uint4*>(p.x) + i);
-    DFT(3);
   }
   __syncthreads();  // S1: barriers initialised, x staged
 
@@ -380,12 +329,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (lane == 0) s_xsum[g] = s;
     }
-    DFT(4);
     if (!mbar_wait(bar_router, 0)) {
       set_status(p.status, DEV_TIMEOUT);
       mi->ok = 0;
     }
-    DFT(5);
     for (int g = warp; g < G; g += kDfWarps) {
       const uint2 xv = *reinterpret_cast<const uint2*>(s_x + g * kGroup + 4 * lane);
       const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
@@ -421,7 +368,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       const int e = r0 + r;
       if (lane == 0) p.logits[e] = s + (p.router_bias ? p.router_bias[e] : 0.f);
     }
-    DFT(6);
   }
   __syncthreads();  // S2: this CTA's logits are written
 
@@ -437,9 +383,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         if (lane == 0) set_status(p.status, DEV_TIMEOUT);
         return;
       }
-#ifdef MOE_TRACE
-      if (warp == 0 && b == mi->first_routed) DFT(13);
-#endif
       const uint8_t* tile = smem + (size_t)b * L.tile_bytes;
       const uint16_t* scales = reinterpret_cast<const uint16_t*>(tile + 2 * kDfRows * rowb_up);
       float* red_b = red + (size_t)b * 2 * G * kDfRows;
@@ -467,12 +410,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
   if (producer) {
     if (lane == 0) {
       s_arrived = gbar_arrive(gbar);
-      DFTP(7);
-      if (mi->ok && !gbar_wait(gbar, s_arrived)) {
+      if (mi->ok && (!gbar_wait(gbar, s_arrived) || !test_hold_wait(p.test_ctl))) {
         set_status(p.status, DEV_TIMEOUT);
         mi->ok = 0;
       }
-      DFTP(8);
     }
     __syncwarp();  // the warp reaches the CTA barrier converged
   } else if (mi->ok) {
@@ -491,7 +432,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     const int n_chunks = (E + 31) / 32;
     const int kk = min(k, 32);
     uint32_t* cand = reinterpret_cast<uint32_t*>(smem + L.off_cand);  // [chunk][kk] key, idx
-    DFT(9);
     for (int ch = warp; ch < n_chunks; ch += kDfWarps) {
       const int e = ch * 32 + lane;
       const uint32_t key = (e < E) ? order_key(__ldcg(p.logits + e)) : 0u;
@@ -507,15 +447,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       }
     }
     named_bar_sync(1, kDfCompute);
-    DFT(10);
     // level 2 (warp 0): the k-th best chunk head bounds the picks from below (the k heads at
     // least as good beat anything it beats), so only candidates it does not beat remain;
     // they are ranked among themselves with shuffles (their overall rank: whatever beats a
     // remaining candidate remains too). More than 32 remaining (heavy ties): a table scan.
-#ifdef MOE_TRACE
-    for (int rep = 0; rep < 2; ++rep) {
-      if (rep == 1) DFT(23);
-#endif
     if (warp == 0) {
       auto beats = [](uint32_t ka, uint32_t ia, uint32_t kb, uint32_t ib) {
         return ka > kb || (ka == kb && ia < ib);
@@ -581,9 +516,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         }
       }
     }
-#ifdef MOE_TRACE
-    }
-#endif
     named_bar_sync(1, kDfCompute);
     if (warp == 0) {
       const uint32_t my_key = (lane < k) ? reinterpret_cast<const uint32_t*>(mi->gate)[lane] : 0u;
@@ -594,7 +526,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
       __syncwarp();
       if (lane < k) mi->gate[lane] = z / tot;
-      DFT(11);
     }
   }
   __syncthreads();  // S4: the routing decision
@@ -627,7 +558,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         }
       }
       if (lane == 0) mi->armed_tiles = mi->n_tiles;
-      if (lane == 0) DFTP(12);
       __syncwarp();
       // the routed down rows this CTA will need, into L2 behind the gate/up requests
       for (int i = lane; i < mi->n_units; i += 32) {
@@ -657,7 +587,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       }
     }
     gate_up_items(mi->first_routed, mi->n_tiles);
-    DFT(14);
   }
   __syncthreads();  // S5: every gate/up product of this CTA is in red; tile buffers are free
 
@@ -678,7 +607,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         bulk_g2s(dst + wbytes, bk.s[2] + row * Gf, sbytes, &bar_unit[i]);
       }
       if (lane == 0) mi->armed_units = mi->n_units;
-      if (lane == 0) DFTP(16);
     }
     __syncwarp();
   } else if (ok1) {
@@ -695,7 +623,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       const float hv = gs / (1.f + expf(-gs)) * us;
       p.h[(size_t)mi->tile_slot[b] * f + (size_t)mi->tile_rt[b] * kDfRows + r] = f32_to_bf16_rn(hv);
     }
-    DFT(15);
   }
   __syncthreads();  // S6: h of this CTA written
 
@@ -704,12 +631,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     // every CTA arrives at every barrier, failed or not, so the word stays consistent
     if (lane == 0) {
       s_arrived = gbar_arrive(gbar);
-      DFTP(17);
       if (ok1 && !gbar_wait(gbar, s_arrived)) {
         set_status(p.status, DEV_TIMEOUT);
         mi->ok = 0;
       }
-      DFTP(18);
       if (mi->ok) {  // every h row of the call, into shared memory in one request
         mbar_arrive_expect_tx(bar_h, (uint32_t)S * f * 2);
         mi->armed_h = 1;
@@ -721,7 +646,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     if (mi->ok)
       for (int s = lane; s < S; s += 32)
         bulk_g2s(smem + L.off_h + (size_t)s * f * 2, p.h + (size_t)s * f, f * 2, bar_h);
-    if (lane == 0) DFTP(19);
     __syncwarp();
   }
   __syncthreads();  // S7: the B2 verdict
@@ -811,14 +735,12 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         out[nn] = f32_to_bf16_rn(acc);
       }
     }
-    if (lane == 0) DFTP(24);
     __syncwarp();
   } else {
     bool ready = false;
     if (ok2) {
       ready = warp_wait(bar_h);
       if (!ready && lane == 0) set_status(p.status, DEV_TIMEOUT);
-      DFT(20);
       // h rows -> fragment order in place, and their per-group sums (a half-warp a group:
       // each lane one 8-value chunk, then a fixed tree over the 16 chunks)
       const int n_groups = S * Gf;
@@ -853,9 +775,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       }
     }
     named_bar_sync(2, kDfThreads);
-    DFT(21);
     if (ok2 && ready) down_items(mi->n_split, mi->n_units);  // pass B
-    DFT(22);
     named_bar_sync(1, kDfCompute);
     if (ok2) {
       // y of every whole-tile unit row into red's first row of the unit (in place: a row's
@@ -878,13 +798,9 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         if (p.has_shared) acc += yt[0];
         out[(size_t)mi->unit_rt[mi->n_split + t * S] * kDfRows + r] = f32_to_bf16_rn(acc);
       }
-      DFT(25);
     }
   }
   __syncthreads();
-#ifdef MOE_TRACE
-  if (tid == 0 && blockIdx.x < 160) g_dftrace[blockIdx.x][27] = clock64();
-#endif
 
   // ---------------------------------------------------------------- drain
   // No copy may land after the CTA ends: wait (boundedly) for every one that was issued.

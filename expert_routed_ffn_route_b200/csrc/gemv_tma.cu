@@ -25,13 +25,7 @@
 
 namespace moe {
 
-#ifdef MOE_TRACE
-__device__ long long g_trace[2][160][64];
-#define TRACE(slot) \
-  do { if (ctid == 0 && blockIdx.x < 160 && (slot) < 64) g_trace[GATE_UP ? 0 : 1][blockIdx.x][(slot)] = clock64(); } while (0)
-#else
 #define TRACE(slot) do {} while (0)
-#endif
 
 constexpr int kCons = 16;                    // consumer warps
 constexpr int kTmaThreads = 32 * (kCons + 1);  // + one producer warp
@@ -141,14 +135,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
   volatile int* flag = reinterpret_cast<volatile int*>(smem + L.flag_off);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#ifdef MOE_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 160) {
-    unsigned long long gt;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt));
-    g_trace[GATE_UP ? 0 : 1][blockIdx.x][61] = (long long)gt;
-    g_trace[GATE_UP ? 0 : 1][blockIdx.x][62] = clock64();
-  }
-#endif
   if (threadIdx.x == 0) {
     for (int s = 0; s < Sh::NS; ++s) {
       mbar_init(&full[s], 1);
@@ -158,9 +144,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
     fence_barrier_init();
   }
   __syncthreads();
-  KT_ENTRY(GATE_UP ? 2 : 3);
   pdl_wait();     // plan and activations come from the preceding kernels
-  KT_READY(GATE_UP ? 2 : 3);
 
   const int n_active = p.active[0];
   const int n_rowtiles = N / Sh::ROWS;
@@ -202,10 +186,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
 
   // -------------------------------------------------------------- consumers
   const int ctid = threadIdx.x;  // 0 .. 255
-#ifdef MOE_TRACE
-  int tr = 0;
-  TRACE(tr++);
-#endif
   const int rt = warp / Sh::KS, ks = warp % Sh::KS;
   const int grp = lane >> 2, q4 = lane & 3;
   int staged_slot = -1, staged_c0 = -1;
@@ -218,9 +198,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
     const bool pre = (staged_slot != t.slot || staged_c0 != 0);
     if (pre) stage_tile_rows<GATE_UP>(p, t, 0, K, xs, S, xsum, ctid);
     if (ctid == 0) flag[1] = mbar_wait(&full[s], u & 1) ? 1 : 0;
-#ifdef MOE_TRACE
-    TRACE(tr++);
-#endif
     named_bar_sync(1, 32 * kCons);
     if (!flag[1]) {
       if (ctid == 0) set_status(p.status, DEV_TIMEOUT);
@@ -239,9 +216,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
         named_bar_sync(1, 32 * kCons);  // everyone is done with the previous rows
         stage_tile_rows<GATE_UP>(p, t, c0, K, xs, S, xsum, ctid);
         named_bar_sync(1, 32 * kCons);
-#ifdef MOE_TRACE
-        TRACE(tr++);
-#endif
         staged_slot = t.slot;
         staged_c0 = c0;
       }
@@ -305,7 +279,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
-  if (ctid == 0) KT_EXIT(GATE_UP ? 2 : 3);
   pdl_trigger();  // dependents start as this CTA finishes (see route_fused.cu)
 }
 
@@ -350,11 +323,6 @@ static cudaError_t launch_tma(const Plan& p, cudaStream_t st, bool pdl) {
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-#ifdef MOE_TRACE
-extern "C" __attribute__((visibility("default"))) int moe_trace_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_trace, sizeof(g_trace));
-}
-#endif
 
 bool tma_gemv_supported(const Plan& p) {
   if (p.routed.fmt != 4 || (p.has_shared && p.shared.fmt != 4)) return false;

@@ -111,10 +111,11 @@ Plan make_plan(const moe_layer* L, void* ws) {
   p.router_bias = L->router_bias;
   p.routed = to_bank(L->routed);
   p.shared = to_bank(L->shared);
-  p.status = reinterpret_cast<int32_t*>(b + w.status);
-  p.ticket = reinterpret_cast<int32_t*>(b + w.status + 16);
-  p.gbar = reinterpret_cast<uint32_t*>(b + w.status + 32);
-  p.tile_cnt = reinterpret_cast<int32_t*>(b + w.status + kAlign);
+  p.status = reinterpret_cast<int32_t*>(b + w.status + kSyncStatus);
+  p.ticket = reinterpret_cast<int32_t*>(b + w.status + kSyncTicket);
+  p.gbar = reinterpret_cast<uint32_t*>(b + w.status + kSyncGbar);
+  p.test_ctl = reinterpret_cast<const int32_t*>(b + w.status + kSyncTest);
+  p.tile_cnt = reinterpret_cast<int32_t*>(b + w.status + kSyncTiles);
   p.logits = reinterpret_cast<float*>(b + w.logits);
   p.topk_idx = reinterpret_cast<int32_t*>(b + w.topk_idx);
   p.topk_w = reinterpret_cast<float*>(b + w.topk_w);
@@ -384,6 +385,20 @@ int32_t moe_launches_per_call(const moe_layer* L) {
   int ffn = use_tc(p) ? 3 : 2;  // (+ gather/schedule) gate/up, down
   if (p.has_shared && p.shared.fmt != p.routed.fmt) ffn += 2;  // each GEMM once per bank
   return route + ffn + 1;       // + combine
+}
+
+moe_status moe_test_inject_hold(const moe_layer* L, void* ws, size_t ws_bytes, int32_t hold,
+                                int32_t budget_cycles, moe_stream_t stream) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (budget_cycles < 0) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, ws, ws_bytes)) != MOE_OK) return s;
+  int32_t* dev = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + layout(L).status + kSyncTest);
+  const int32_t words[2] = {hold ? 1 : 0, budget_cycles};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // pageable source: the call returns once the words are staged, so a stack array is fine
+  MOE_TRY(cudaMemcpyAsync(dev, words, sizeof(words), cudaMemcpyHostToDevice, st));
+  return MOE_OK;
 }
 
 moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,

@@ -80,6 +80,60 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ grid barrier
+
+// Grid-wide barrier on one 32-bit word whose low 31 bits are zero between barriers (the
+// workspace starts zeroed). Every CTA adds to the word exactly once per barrier; CTA 0 adds
+// 2^31 - (grid - 1) and the others 1, so the top bit flips exactly when the last CTA
+// arrives, in whatever order they come, and the low bits are zero again afterwards. A CTA is
+// through once it sees the top bit differ from the value it found on arrival. A CTA that
+// gave up waiting still left its arrival behind, so a late arrival completes its own
+// barrier and never leaks into the next one; the grid size may change from call to call.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// Arrival: a release (this CTA's writes, ordered before it by the CTA barrier the caller
+// has passed, become visible to every CTA that sees the arrival).
+__device__ __forceinline__ uint32_t gbar_arrive(uint32_t* bar) {
+  const uint32_t add = (blockIdx.x == 0) ? (0x80000000u - (gridDim.x - 1)) : 1u;
+  fence_acq_rel_gpu();
+  return atomicAdd(bar, add);
+}
+
+// Waits (boundedly) until the barrier `arrived` (the value gbar_arrive returned) completes.
+__device__ __forceinline__ bool gbar_wait(const uint32_t* bar, uint32_t arrived) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t now;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(bar) : "memory");
+    if ((now ^ arrived) & 0x80000000u) break;
+    if (clock64() - t0 > kWaitCycles) return false;
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ failure injection
+
+// Test hook: while the workspace's hold word (test_ctl[0]) is nonzero, the kernels that
+// check it wait for it to return to zero, which nothing does during the call, so the wait
+// runs out after test_ctl[1] clock cycles (kWaitCycles when that is zero) and reports
+// DEV_TIMEOUT, exactly as a wait on a peer that never arrives would. Returns false on that
+// timeout; true at once when the hold word is zero (the normal case: one load).
+__device__ __forceinline__ bool test_hold_wait(const int32_t* test_ctl) {
+  if (!test_ctl) return true;
+  if (__ldcg(test_ctl) == 0) return true;
+  const int32_t budget = __ldcg(test_ctl + 1);
+  const long long limit = budget > 0 ? (long long)budget : kWaitCycles;
+  const long long t0 = clock64();
+  while (*(volatile const int32_t*)test_ctl != 0) {
+    if (clock64() - t0 > limit) return false;
+    __nanosleep(64);
+  }
+  return true;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -89,22 +143,5 @@ __device__ __forceinline__ void named_bar_arrive(int id, int threads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-#ifdef MOE_TRACE
-// Kernel timeline (trace builds only): per kernel id, earliest entry, earliest and latest
-// return from the dependency wait, latest exit, in globaltimer nanoseconds.
-extern __device__ unsigned long long g_ktime[8][4];
-__device__ __forceinline__ unsigned long long gtime() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-#define KT_ENTRY(id) do { if (threadIdx.x == 0) atomicMin(&g_ktime[id][0], gtime()); } while (0)
-#define KT_READY(id) do { if (threadIdx.x == 0) { unsigned long long _t = gtime(); atomicMin(&g_ktime[id][1], _t); atomicMax(&g_ktime[id][2], _t); } } while (0)
-#define KT_EXIT(id) do { atomicMax(&g_ktime[id][3], gtime()); } while (0)
-#else
-#define KT_ENTRY(id) do {} while (0)
-#define KT_READY(id) do {} while (0)
-#define KT_EXIT(id) do {} while (0)
-#endif
 
 }  // namespace moe

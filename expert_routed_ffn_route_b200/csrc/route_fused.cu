@@ -6,7 +6,8 @@
 // registers. Phase 2 (CTAs 0 .. T-1, once every CTA has counted itself in a ticket after a
 // memory fence): CTA t ranks token t (stable top-k and gates). Phase 3 (the last of those to
 // finish, found with a second ticket): the expert-major plan and the active-expert list,
-// then both tickets are cleared for the next call.
+// then the second ticket is cleared for the next call (the first is a grid barrier word
+// that returns to its start value by itself).
 //
 // Rules followed: deterministic stable top-k, ties to the lower expert index
 // (Qwen3.8-Flash-Next-Dual-GPU README, "Independent decode lane"); gates = softmax over the
@@ -18,25 +19,6 @@
 
 namespace moe {
 
-#ifdef MOE_TRACE
-__device__ unsigned long long g_ktime[8][4];
-extern "C" __attribute__((visibility("default"))) int moe_ktime_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_ktime, sizeof(g_ktime));
-}
-extern "C" __attribute__((visibility("default"))) int moe_ktime_reset() {
-  unsigned long long h[8][4];
-  for (int i = 0; i < 8; ++i) { h[i][0] = h[i][1] = ~0ull; h[i][2] = h[i][3] = 0; }
-  return (int)cudaMemcpyToSymbol(g_ktime, h, sizeof(h));
-}
-__device__ long long g_rtrace[160][8];
-#define RTRACE(slot) \
-  do { if (threadIdx.x == 0 && blockIdx.x < 160) g_rtrace[blockIdx.x][(slot)] = clock64(); } while (0)
-extern "C" __attribute__((visibility("default"))) int moe_rtrace_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_rtrace, sizeof(g_rtrace));
-}
-#else
-#define RTRACE(slot) do {} while (0)
-#endif
 
 constexpr int kRFWarps = 4;
 constexpr int kRFThreads = 32 * kRFWarps;
@@ -51,17 +33,7 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
   __shared__ int s_wsum[kRFWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int T = p.T, E = p.E, d = p.d, k = p.k;
-#ifdef MOE_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 160) {
-    unsigned long long gt;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt));
-    g_rtrace[blockIdx.x][7] = (long long)gt;
-  }
-#endif
-  RTRACE(0);
-  KT_ENTRY(0);
   pdl_wait();
-  KT_READY(0);
 
   // ---------------------------------------------------------------- logits
   // A lane owns 16-byte pieces c = lane + 32 i of the router row (d <= 8192: i < 32); the
@@ -123,35 +95,28 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
   }
 
   // ---------------------------------------------------------------- tickets
-  // Every CTA publishes its logits and counts itself in ticket[0]; CTAs T.. leave. CTA t < T
-  // waits, boundedly, until all CTAs have counted themselves (all CTAs of this grid are
-  // resident together: gridDim = max(E / 4, T) <= 256 small CTAs), ranks token
-  // t, and counts itself in ticket[1]; the last one builds the plan. After a timeout the
-  // status word is set and the CTA goes on (its picks are then unreliable, but every ticket
-  // is still met and cleared).
-  RTRACE(1);
+  // Every CTA publishes its logits and arrives at a grid barrier on ticket[0] (the flip-bit
+  // barrier of pipeline.cuh); CTAs T.. leave. CTA t < T waits, boundedly, for the barrier
+  // (all CTAs of this grid are resident together: gridDim = max(E / 4, T) <= 256 small
+  // CTAs), ranks token t, and counts itself in ticket[1]; the last one builds the plan and
+  // clears ticket[1]. After a timeout the status word is set and the CTA goes on (its picks
+  // are then unreliable); every CTA has arrived all the same, so the barrier word is
+  // consistent for the next call.
+  __shared__ uint32_t s_arrived;
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) atomicAdd(&ticket[0], 1);
+  if (threadIdx.x == 0) s_arrived = gbar_arrive(reinterpret_cast<uint32_t*>(&ticket[0]));
   if ((int)blockIdx.x >= T) {
-    if (threadIdx.x == 0) KT_EXIT(0);
     return;  // an exited CTA counts as having released its dependents
   }
   if (threadIdx.x == 0) {
-    const long long t0 = clock64();
-    while (*(volatile int*)&ticket[0] < (int)gridDim.x) {
-      if (clock64() - t0 > kWaitCycles) {
-        set_status(p.status, DEV_TIMEOUT);
-        break;
-      }
-    }
+    if (!gbar_wait(reinterpret_cast<const uint32_t*>(&ticket[0]), s_arrived))
+      set_status(p.status, DEV_TIMEOUT);
+    else if (!test_hold_wait(p.test_ctl))
+      set_status(p.status, DEV_TIMEOUT);
   }
   __syncthreads();
-  RTRACE(2);
   __threadfence();
-#ifdef MOE_TRACE
-  long long c_fence = clock64();
-#endif
 
   // ---------------------------------------------------------------- top-k and gates
   if (warp == 0) {
@@ -166,16 +131,11 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
       p.topk_w[(size_t)t * k + lane] = g;
     }
   }
-  RTRACE(3);
-#ifdef MOE_TRACE
-  if (threadIdx.x == 0) g_ktime[5][1] = clock64() - c_fence;
-#endif
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = (atomicAdd(&ticket[1], 1) == T - 1);
   __syncthreads();
   if (!s_last) {
-    if (threadIdx.x == 0) KT_EXIT(0);
     return;
   }
   __threadfence();
@@ -274,19 +234,11 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
     }
   }
   __syncthreads();
-  RTRACE(4);
-#ifdef MOE_TRACE
-  if (threadIdx.x == 0) g_ktime[6][0] = clock64() - c_fence;
-#endif
   __syncthreads();
-  if (threadIdx.x == 0) {
-    ticket[0] = 0;
-    ticket[1] = 0;
-  }
+  if (threadIdx.x == 0) ticket[1] = 0;
   // The next kernel is released only now: kernels whose CTAs wait early for this one share
   // the SMs and slow the last CTA down.
   pdl_trigger();
-  if (threadIdx.x == 0) KT_EXIT(1);
 }
 
 bool route_fused_supported(const Plan& p) { return p.T <= kRFMaxT && p.E <= kMaxE; }

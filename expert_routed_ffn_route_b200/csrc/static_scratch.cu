@@ -40,11 +40,29 @@ extern "C" moe_status moe_layer_forward_static(const moe_layer* L, const void* x
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_TOO_LARGE;
   void* ws = nullptr;
   if ((s = scratch_address(&ws)) != MOE_OK) return s;
-  // the synchronisation block at the start of the workspace (status word, routing ticket,
-  // barrier word, tile counters) begins at zero
-  if (cudaMemsetAsync(ws, 0, moe::sync_bytes(L->d), reinterpret_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  // the synchronisation block after the status word (routing tickets, barrier word,
+  // failure-injection words, tile counters) begins at zero; the status word itself is kept
+  // until moe_static_device_status reads it (the array starts zeroed at load)
+  uint8_t* sync = static_cast<uint8_t*>(ws) + moe::kSyncTicket;
+  if (cudaMemsetAsync(sync, 0, moe::sync_bytes(L->d) - moe::kSyncTicket,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
   return moe_layer_forward(L, x, out, nullptr, nullptr, nullptr, nullptr, ws,
                            MOE_STATIC_SCRATCH_BYTES, stream);
+}
+
+extern "C" moe_status moe_static_device_status(int32_t* code, moe_stream_t stream) {
+  if (!code) return MOE_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  moe_status s = scratch_address(&ws);
+  if (s != MOE_OK) return s;
+  int32_t* dev = static_cast<int32_t*>(ws) + moe::kSyncStatus / sizeof(int32_t);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, dev, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess ||
+      cudaMemsetAsync(dev, 0, sizeof(int32_t), st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *code = (h == moe::DEV_OK) ? MOE_OK : (h == moe::DEV_TIMEOUT ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE);
+  return MOE_OK;
 }

@@ -47,37 +47,6 @@
 
 namespace moe {
 
-#ifdef MOE_TRACE
-__device__ long long g_tct[2][4][16][2];  // [kernel][role][unit][start/end], CTA 0
-#define TCT(role, ui, se) \
-  do { if (blockIdx.x == 0 && (ui) < 16) g_tct[GATE_UP ? 0 : 1][role][ui][se] = clock64(); } while (0)
-__device__ long long g_tcc[2][48][6];  // [kernel][chunk of unit 0][event], CTA 0
-#define TCC(c, ev) \
-  do { if (blockIdx.x == 0 && (c) < 48) g_tcc[GATE_UP ? 0 : 1][c][ev] = clock64(); } while (0)
-__device__ long long g_tcw[2][48][8][3];  // [kernel][chunk][dequant warp][start, waited, arrival]
-#define TCW(c, ev) \
-  do { if (blockIdx.x == 0 && lane == 0 && (c) < 48) g_tcw[GATE_UP ? 0 : 1][c][warp - 2][ev] = clock64(); } while (0)
-__device__ long long g_tcs[2][16][8][2];  // [kernel][weight stage][dequant warp][before, after full_w]
-#define TCS(st, ev) \
-  do { if (blockIdx.x == 0 && lane == 0 && (st) < 16) g_tcs[GATE_UP ? 0 : 1][st][warp - 2][ev] = clock64(); } while (0)
-extern "C" __attribute__((visibility("default"))) int moe_tcs_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_tcs, sizeof(g_tcs));
-}
-extern "C" __attribute__((visibility("default"))) int moe_tcw_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_tcw, sizeof(g_tcw));
-}
-extern "C" __attribute__((visibility("default"))) int moe_tcc_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_tcc, sizeof(g_tcc));
-}
-extern "C" __attribute__((visibility("default"))) int moe_tct_read(void* dst) {
-  return (int)cudaMemcpyFromSymbol(dst, g_tct, sizeof(g_tct));
-}
-#else
-#define TCT(role, ui, se) do {} while (0)
-#define TCC(c, ev) do {} while (0)
-#define TCW(c, ev) do {} while (0)
-#define TCS(st, ev) do {} while (0)
-#endif
 
 constexpr int kTcThreads = 512;  // 16 warps
 constexpr int kDqWarps = 8;       // dequantisers (two threads per weight row)
@@ -547,7 +516,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
         const int src = t.shared ? 1 : 0;
         const int wrow = t.e * N + t.ntile * kTcM;
-        TCT(0, ui, 0);
         if constexpr (FMT != 16) {
           // the unit's group scales: kTcM consecutive rows, one contiguous block per matrix
           const int sbuf = ui & 1;
@@ -583,7 +551,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           fail();
           break;
         }
-        TCT(0, ui, 1);
       }
       // every issued stage lands before the CTA may exit (consumed ones already have)
       for (int j = (it > C::NW ? it - C::NW : 0); j < it; ++j)
@@ -620,13 +587,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       aborted = __any_sync(0xffffffffu, aborted);
       tc_fence_after();
-      TCT(1, tile, 0);
       const uint32_t dacc = tmem + b * 128 + iss * kTcNMax;  // this issuer's accumulator
       for (int c = 0; c < n_chunks; ++c, ++it) {
         const int s = it % C::NX;
         named_bar_sync(1 + s, kReadyThreads);
         tc_fence_after();
-        TCC(it, 1);
         // One descriptor and one TMEM address per chunk; the K steps advance them by
         // constants (32 bytes of B = 2 in the descriptor's address field, 8 columns of A).
         const uint64_t bdesc = umma_desc_sw128(smem_u32(smem + C::X_OFF + s * C::XB));
@@ -637,10 +602,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma_f16_ts_warp(dacc, at + (k0 + kk) * 8, bdesc + (uint64_t)(2 * (k0 + kk)), idesc,
                              (c > 0 || kk > 0) ? 1u : 0u);
         umma_commit_warp(&empty_x[s]);  // releases the activation stage and the A stage
-        TCC(it, 2);
       }
       umma_commit_warp(&acc_full[b]);
-      TCT(1, tile, 1);
     }
     // all issued MMAs complete before TMEM and shared memory are released
     umma_commit_warp(drain);
@@ -666,7 +629,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int u = u_begin + (int)blockIdx.x; u < total; u += gridDim.x, ++ui) {
       const int sbuf = ui & 1;
       aborted = aborted || *abort_flag;
-      if (threadIdx.x == 64) TCT(2, ui, 0);
       if constexpr (FMT != 16) {
         if (!aborted && !mbar_wait(&scale_full[sbuf], (ui >> 1) & 1)) {
           fail();
@@ -679,18 +641,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int sw = it % C::NW;
         // every warp waits for every stage before releasing it (keeps the release phases
         // of the stage in order, also for a group with no chunk in it)
-        TCS(it, 0);
         if (!aborted && !mbar_wait(&full_w[sw], (it / C::NW) & 1)) {
           fail();
           aborted = true;
         }
         aborted = __any_sync(0xffffffffu, aborted);
-        TCS(it, 1);
         const int c_end = min(n_chunks, (cw + 1) * C::SUB);
         for (int c = cw * C::SUB; c < c_end; c += CH, ia += CH) {
           if (((c / CH) & 1) != group) continue;
-          if ((threadIdx.x & 127) == 64) TCC(ia, 3);
-          TCW(ia, 0);
 #pragma unroll
           for (int j = 0; j < CH; ++j) {
             const int a = (ia + j) % C::NA;
@@ -706,8 +664,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           }
           aborted = __any_sync(0xffffffffu, aborted);
-          if ((threadIdx.x & 127) == 64) TCC(ia, 4);
-          TCW(ia, 1);
           if (!aborted) {
 #pragma unroll
             for (int j = 0; j < CH; ++j) {
@@ -729,8 +685,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           tc_fence_before();  // the stores are complete before the arrivals below
           __syncwarp();
-          if ((threadIdx.x & 127) == 64) TCC(ia, 5);
-          TCW(ia, 2);
 #pragma unroll
           for (int j = 0; j < CH; ++j) named_bar_arrive(1 + (ia + j) % C::NA, kReadyThreads);
         }
@@ -741,7 +695,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&scale_empty[sbuf]);
       }
-      if (threadIdx.x == 64) TCT(2, ui, 1);
     }
   } else if (warp == 15) {
     // ------------------------------------------------------------ activation producer
@@ -785,7 +738,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       tc_fence_after();
-      if (threadIdx.x == 320) TCT(3, tile, 0);
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + b * 128;
       const int n = t.ntile * kTcM + row;  // output feature
       // gate/up: where feature n sits in the h row (the K order the down GEMM's bank reads)
@@ -824,7 +776,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
-      if (threadIdx.x == 320) TCT(3, tile, 1);
     }
   }
 

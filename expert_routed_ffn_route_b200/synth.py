@@ -43,7 +43,7 @@ import numpy as np
 __all__ = [
     "LayerConfig", "CONFIGS", "Bank", "LayerInputs", "make_layer", "make_bank",
     "make_router", "make_hidden", "bf16_bits", "bf16_bits_to_f32", "pack_int4",
-    "quantize_groups", "derive_seed", "FMT_BITS",
+    "quantize_groups", "derive_seed", "FMT_BITS", "plant_ties",
 ]
 
 FMT_BITS = {"bf16": 16, "int8": 8, "int4": 4}
@@ -310,7 +310,9 @@ def make_router(cfg: LayerConfig):
     return wr, bias
 
 
-def _margins_ok(logits: np.ndarray, k: int, margin: float) -> np.ndarray:
+def _margins_ok(logits: np.ndarray, k: int, margin: float, ties=None) -> np.ndarray:
+    if ties:
+        return np.array([_margins_ok_ties(row, k, margin, ties) for row in logits], bool)
     kk = min(k + 1, logits.shape[1])
     top = -np.sort(-logits, axis=1)[:, :kk]
     if kk < 2:
@@ -318,10 +320,33 @@ def _margins_ok(logits: np.ndarray, k: int, margin: float) -> np.ndarray:
     return np.all(top[:, :-1] - top[:, 1:] >= margin, axis=1)
 
 
+def _margins_ok_ties(row: np.ndarray, k: int, margin: float, ties) -> bool:
+    """The margin rule with planted tie groups (experts whose logits are equal by
+    construction): each group counts as one entry of its size, and the entries that cover
+    the first k + 1 experts must be ``margin`` apart."""
+    drop = np.zeros(row.size, bool)
+    size = np.ones(row.size, np.int64)
+    for g in ties:
+        g = sorted(int(e) for e in g)
+        drop[g[1:]] = True
+        size[g[0]] = len(g)
+    keep = np.flatnonzero(~drop)
+    order = keep[np.argsort(-row[keep], kind="stable")]
+    covered, vals = 0, []
+    for e in order:
+        vals.append(row[e])
+        covered += size[e]
+        if covered >= k + 1:
+            break
+    v = np.asarray(vals)
+    return bool(np.all(v[:-1] - v[1:] >= margin))
+
+
 def make_hidden(cfg: LayerConfig, wr_bits: np.ndarray, bias, T: int | None = None,
-                stream: str = "x", max_tries: int = 1000) -> np.ndarray:
+                stream: str = "x", max_tries: int = 1000, ties=None) -> np.ndarray:
     """Hidden states [T, d] (bf16 bits), N(0,1), every row redrawn (from its own
-    stream) until its routing margin holds."""
+    stream) until its routing margin holds. ``ties`` lists groups of experts whose logits
+    are planted equal (identical router rows and bias); each group counts once."""
     T = cfg.T if T is None else T
     wrf = bf16_bits_to_f32(wr_bits).astype(np.float64)
     b = np.zeros(cfg.E) if bias is None else bias.astype(np.float64)
@@ -332,7 +357,7 @@ def make_hidden(cfg: LayerConfig, wr_bits: np.ndarray, bias, T: int | None = Non
         rows = np.stack([bf16_bits(_normal((cfg.d,), 1.0, cfg.seed, stream, int(t), tries))
                          for t in pending])
         lg = bf16_bits_to_f32(rows).astype(np.float64) @ wrf.T + b
-        ok = _margins_ok(lg, cfg.k, cfg.margin)
+        ok = _margins_ok(lg, cfg.k, cfg.margin, ties)
         out[pending[ok]] = rows[ok]
         pending = pending[~ok]
         tries += 1
@@ -350,6 +375,20 @@ class LayerInputs:
     routed: Bank
     shared: Bank | None
     extra: dict = field(default_factory=dict)
+
+
+def plant_ties(wr_bits: np.ndarray, bias, groups, lifts):
+    """Router with planted ties: every expert of ``groups[i]`` gets the router row of the
+    group's first expert and the bias ``lifts[i]`` (experts outside the groups keep their
+    rows and get bias 0, or keep the given bias). Identical rows and bias give logits that
+    are equal in any arithmetic that treats the rows alike. Returns (router bits, bias)."""
+    wr = wr_bits.copy()
+    b = np.zeros(wr.shape[0], np.float32) if bias is None else bias.astype(np.float32).copy()
+    for g, lift in zip(groups, lifts):
+        g = [int(e) for e in g]
+        wr[g] = wr[g[0]]
+        b[g] = np.float32(lift)
+    return wr, b
 
 
 def make_layer(cfg: LayerConfig | str, T: int | None = None, routed: Bank | None = None,

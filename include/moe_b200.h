@@ -180,6 +180,20 @@ MOE_API int32_t moe_launches_per_call(const moe_layer* L);
 MOE_API moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,
                              moe_stream_t stream);
 
+/* Failure injection, for tests of the error path: sets (hold != 0) or clears (hold == 0)
+ * the hold word in the workspace's synchronisation block, with a wait budget in SM clock
+ * cycles (0 = the library's normal bound of about two seconds). While the word is set, the
+ * single-kernel 1-token layer (at its first grid barrier) and the fused routing kernel of
+ * calls of up to 32 tokens (after its ticket barrier) wait for the word to return to zero,
+ * which nothing does during a call: the wait runs out after the budget, the kernel records
+ * MOE_ERR_TIMEOUT in the status word (read by moe_device_status), drains its copies and
+ * returns, exactly as when a peer never arrives. Nothing hangs and nothing faults. The
+ * words are written with an asynchronous copy on `stream` (not for use during capture).
+ * Clear the word (or use a fresh workspace) before normal use. */
+MOE_API moe_status moe_test_inject_hold(const moe_layer* L, void* ws, size_t ws_bytes,
+                                        int32_t hold, int32_t budget_cycles,
+                                        moe_stream_t stream);
+
 /* For callers that cannot allocate device memory. Some callers have no way to call
  * cudaMalloc when the layer runs: code running inside a stream-ordered region whose
  * allocator is owned by someone else, plug-ins that are handed a stream but no allocator,
@@ -196,7 +210,8 @@ MOE_API moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_byt
  *   - The first call on a device looks up the buffer's device address (once per device);
  *     make that first call before capturing a stream into a CUDA graph.
  *   - Every call on a device shares the one buffer, and it keeps the previous call's
- *     contents (the call clears the words that must start at zero). Calls that can run at
+ *     contents (the call clears the words that must start at zero, except the status
+ *     word, which moe_static_device_status reads and clears). Calls that can run at
  *     the same time on one device (different streams, or different host threads without
  *     ordering) race on it and give wrong results; order them on one stream.
  *   - x and out as for moe_layer_forward; the routing outputs are not returned.
@@ -205,6 +220,14 @@ MOE_API moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_byt
 #define MOE_STATIC_SCRATCH_BYTES (16u << 20)
 MOE_API moe_status moe_layer_forward_static(const moe_layer* L, const void* x, void* out,
                                             moe_stream_t stream);
+
+/* The device status word of the built-in scratch used by moe_layer_forward_static on the
+ * current device (the counterpart of moe_device_status for that entry point): synchronises
+ * `stream`, writes MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE to *code and clears the word.
+ * A static call leaves the word as its kernels set it (it does not clear it), so an error
+ * of any call since the last read is reported here. Allocates nothing. Like the first static
+ * call, the first call of this function on a device looks up the buffer's address. */
+MOE_API moe_status moe_static_device_status(int32_t* code, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,7 @@ NVFP4, as NVIDIA defines it (the pages name the format but do not spell it out):
     (m / 8 * 2^-6); the code with all exponent and mantissa bits set is NaN; largest 448.
   - one float32 scale per tensor. value = e2m1 * e4m3 * scale.
 
-Readings taken where neither the pages nor the format fix a step (listed in the design doc too):
+Readings taken where neither the pages nor the format fix a step:
   N1  weights: encoded once by the generator, block scale = E4M3(amax_block / (6 g)) with
       g = amax(matrix) / (6 * 448), element = E2M1(w / (block scale * g)), both rounded to
       nearest even, elements saturating at 6 (the usual NVFP4 recipe).

@@ -11,20 +11,11 @@ import pytest
 
 from oracle import moe_oracle as O
 from expert_routed_ffn_route_b200 import synth
-from conftest import bank_dict, out_tol, output_excess
+from conftest import out_tol, output_excess
+from gpu_helpers import bf16_to_np, check_layer, oracle_run, plan_edge_tokens, to_dev_x
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
-
-GATE_TOL = 1e-5
-
-
-def to_dev_x(x_bits):
-    return torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
-
-
-def bf16_to_np(t):
-    return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
 @pytest.fixture(scope="module")
@@ -34,64 +25,6 @@ def B():
         pytest.skip("no GPU")
     binding.load_library()
     return binding
-
-
-def oracle_run(L: synth.LayerInputs, tokens=None, x=None):
-    x = L.x if x is None else x
-    return O.layer_forward(x, L.router_w, L.router_bias, bank_dict(L.routed),
-                           bank_dict(L.shared), L.cfg.k, tokens=tokens)
-
-
-def check_layer(B, dl, L, x_bits, path, sample=None, check_stages=True):
-    T = x_bits.shape[0]
-    desc = dl.descriptor(T, path)
-    ws = B.alloc_workspace(desc)
-    x = to_dev_x(x_bits)
-    idx = torch.empty((T, L.cfg.k), dtype=torch.int32, device="cuda")
-    w = torch.empty((T, L.cfg.k), dtype=torch.float32, device="cuda")
-    offs = torch.empty(L.cfg.E + 1, dtype=torch.int32, device="cuda")
-    perm = torch.empty(T * L.cfg.k, dtype=torch.int32, device="cuda")
-    out = B.layer_forward(desc, x, ws, topk_idx=idx, topk_w=w, offsets=offs, perm=perm)
-    out2 = B.layer_forward(desc, x, ws)
-    torch.cuda.synchronize()
-    assert B.device_status(desc, ws) == 0
-    assert torch.equal(out.view(torch.int16), out2.view(torch.int16)), "not deterministic"
-
-    tokens = np.arange(T) if sample is None else np.asarray(sample)
-    ref = oracle_run(L, tokens=tokens, x=x_bits)
-    assert np.array_equal(idx.cpu().numpy(), ref["idx"]), "expert indices differ"
-    np.testing.assert_allclose(w.cpu().numpy(), ref["gates"], rtol=0, atol=GATE_TOL)
-    assert np.array_equal(offs.cpu().numpy(), ref["offsets"])
-    assert np.array_equal(perm.cpu().numpy(), ref["perm"])
-    got = O.widen_bf16(bf16_to_np(out))[tokens]
-    err = float(output_excess(got, ref["out"]).max())
-    raw = float(np.abs(got - ref["out"]).max())
-    print(f"[{L.cfg.name} T={T} {path}] max|d| {raw:.3e}, beyond bf16 rounding {err:.3e}, "
-          f"bound {out_tol(ref['out']):.3e}")
-    assert err <= out_tol(ref["out"]), f"max excess {err} > {out_tol(ref['out'])}"
-
-    if check_stages:
-        # the four stage entry points give the multi-kernel call's result bit for bit (the
-        # single-kernel 1-token layer sums in another order: there, both meet the oracle)
-        i2, w2 = B.route(desc, x, ws)
-        o2, p2, inv2 = B.permute(desc, i2, ws)
-        ya, ys = B.grouped_ffn(desc, x, o2, p2, ws, has_shared=dl.has_shared)
-        out3 = B.combine(desc, ya, ys, inv2, w2)
-        torch.cuda.synchronize()
-        one_kernel = B.launches_per_call(desc) == 1
-        assert torch.equal(i2, idx)
-        if one_kernel:  # logits summed in another order: gates agree to the gate tolerance
-            np.testing.assert_allclose(w2.cpu().numpy(), w.cpu().numpy(), rtol=0, atol=GATE_TOL)
-        else:
-            assert torch.equal(w2, w)
-        assert torch.equal(o2, offs) and torch.equal(p2, perm)
-        assert np.array_equal(inv2.cpu().numpy(), ref["inv"])
-        if one_kernel:
-            got3 = O.widen_bf16(bf16_to_np(out3))[tokens]
-            assert float(output_excess(got3, ref["out"]).max()) <= out_tol(ref["out"])
-        else:
-            assert torch.equal(out3.view(torch.int16), out.view(torch.int16))
-    return err
 
 
 # ------------------------------------------------------------------ small shapes
@@ -154,14 +87,19 @@ def int4_bank(B):
     return routed, shared
 
 
-@pytest.mark.parametrize("name,sample", [("decode", None), ("verify16", None),
-                                         ("verify32", [0, 7, 31]),
-                                         ("prefill", [0, 1, 255, 511])])
-def test_full_size_int4(B, int4_bank, name, sample):
+@pytest.mark.parametrize("name", ["decode", "verify16", "verify32", "prefill"])
+def test_full_size_int4(B, int4_bank, name):
+    """Full-size int4 workloads in the launch configuration the bench times (path auto).
+    Every output row of the decode and verify calls is compared; at prefill, 128 rows:
+    the edges of the units of the 8 most loaded experts and a seeded random draw."""
     cfg = synth.CONFIGS[name]
     routed, shared = int4_bank
     L = synth.make_layer(cfg, routed=routed, shared=shared)
     dl = B.DeviceLayer(L)
+    sample = None
+    if cfg.T > 32:
+        sample = plan_edge_tokens(L, n_hot=8, n_total=128, seed=1)
+        assert len(sample) == 128
     check_layer(B, dl, L, L.x, "auto", sample=sample, check_stages=(cfg.T <= 32))
 
 
@@ -181,10 +119,16 @@ def test_full_size_decode_paths(B, int4_bank, path, shared):
 
 
 def test_full_size_long_int8(B):
+    """The long Zipf-skewed int8 workload: 256 output rows, including the first row of each
+    of the 5 most loaded experts and the first and last rows of their last (ragged)
+    tensor-core unit, the rest a seeded random draw (every hot expert's units alternate
+    between the two accumulator buffers of the gate/up GEMM)."""
     cfg = synth.CONFIGS["long"]
     L = synth.make_layer(cfg)
     dl = B.DeviceLayer(L)
-    check_layer(B, dl, L, L.x, "auto", sample=[0, 1, 2047, 4095], check_stages=False)
+    sample = plan_edge_tokens(L, n_hot=5, n_total=256, seed=2)
+    assert len(sample) == 256
+    check_layer(B, dl, L, L.x, "auto", sample=sample, check_stages=False)
 
 
 # ------------------------------------------------------------------ errors
