@@ -156,9 +156,9 @@ struct Plan {
   int32_t* status;
   int32_t* ticket;     // [2]: the fused routing kernel's grid-barrier word and its ranking
                        // counter (zero between calls)
-  uint32_t* gbar;      // grid-barrier word of the single-kernel 1-token path (any value)
   int32_t* tile_cnt;   // [d / 16] per-output-tile arrival counters, zero between calls
   const int32_t* test_ctl;  // failure injection: [0] hold word, [1] wait budget (cycles)
+  uint32_t* gbar;      // grid-barrier word of the single-kernel 1-token layer
   uint16_t* xg;        // tensor-core path: fp16 x rows in grouped order, then the shared
                        // expert's rows [(T*k + T)][d]
   int32_t* tc_sched;   // tensor-core path: per-slot schedule (TcSched view)
@@ -177,8 +177,9 @@ struct TcSched {
 };
 
 // The synchronisation block at the start of the workspace: status word (offset 0), routing
-// tickets (16, 20), grid-barrier word (32), the failure-injection words (64: hold, 68: wait
-// budget; zero in normal use), then one arrival counter per 16-row output tile (256).
+// tickets (16, 20), the single-kernel layer's grid-barrier word (32), the failure-injection
+// words (64: hold, 68: wait budget; zero in normal use), then one arrival counter per 16-row
+// output tile (256).
 constexpr size_t kSyncStatus = 0, kSyncTicket = 16, kSyncGbar = 32, kSyncTest = 64,
                  kSyncTiles = 256;
 inline size_t sync_bytes(int d) { return 256 + (size_t)4 * (d / 16); }
@@ -209,8 +210,7 @@ cudaError_t launch_tc_gate_up(const Plan& p, const TcSched& S, const uint16_t* x
 cudaError_t launch_tc_down(const Plan& p, const TcSched& S, cudaStream_t st);
 // the whole layer of a 1-token call in one persistent kernel (decode_fused.cu)
 bool decode_fused_supported(const Plan& p);
-cudaError_t launch_decode_fused(const Plan& p, void* out, uint32_t* gbar, int32_t* tile_cnt,
-                                cudaStream_t st);
+cudaError_t launch_decode_fused(const Plan& p, void* out, cudaStream_t st);
 // router + top-k + plan in one launch (T <= 32)
 bool route_fused_supported(const Plan& p);
 cudaError_t launch_route_fused(const Plan& p, int32_t* ticket, cudaStream_t st);

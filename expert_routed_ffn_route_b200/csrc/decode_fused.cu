@@ -856,8 +856,9 @@ bool decode_fused_supported(const Plan& p) {
   return true;
 }
 
-cudaError_t launch_decode_fused(const Plan& p, void* out, uint32_t* gbar, int32_t* tile_cnt,
-                                cudaStream_t st) {
+cudaError_t launch_decode_fused(const Plan& p, void* out, cudaStream_t st) {
+  uint32_t* gbar = p.gbar;
+  int32_t* tile_cnt = p.tile_cnt;
   int sms = 0;
   cudaError_t err = df_sms(&sms);
   if (err != cudaSuccess) return err;

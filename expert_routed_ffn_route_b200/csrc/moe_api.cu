@@ -341,7 +341,7 @@ moe_status moe_layer_forward_marked(const moe_layer* L, const void* x, void* out
   MOE_TRY(mark(0));
   if (use_fused(p)) {
     // one kernel: every stage mark after it
-    MOE_TRY(launch_decode_fused(p, out, p.gbar, p.tile_cnt, st));
+    MOE_TRY(launch_decode_fused(p, out, st));
     for (int i = 1; i < MOE_N_MARKS; ++i) MOE_TRY(mark(i));
     return MOE_OK;
   }

@@ -40,9 +40,9 @@ extern "C" moe_status moe_layer_forward_static(const moe_layer* L, const void* x
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_TOO_LARGE;
   void* ws = nullptr;
   if ((s = scratch_address(&ws)) != MOE_OK) return s;
-  // the synchronisation block after the status word (routing tickets, barrier word,
-  // failure-injection words, tile counters) begins at zero; the status word itself is kept
-  // until moe_static_device_status reads it (the array starts zeroed at load)
+  // the synchronisation block from the routing tickets on (tickets, barrier word,
+  // failure-injection words, h counters, tile counters) begins at zero; the status word is
+  // kept until moe_static_device_status reads it (the array starts zeroed at load)
   uint8_t* sync = static_cast<uint8_t*>(ws) + moe::kSyncTicket;
   if (cudaMemsetAsync(sync, 0, moe::sync_bytes(L->d) - moe::kSyncTicket,
                       reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
