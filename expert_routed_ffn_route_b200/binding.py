@@ -13,7 +13,7 @@ import numpy as np
 
 from . import _build
 
-FMT_CODE = {"bf16": 16, "int8": 8, "int4": 4}
+FMT_CODE = {"bf16": 16, "int8": 8, "int4": 4, "nvfp4": 41}
 PATH_CODE = {"auto": 0, "gemv": 1, "tc": 2, "fused": 3}
 N_MARKS = 6
 
@@ -32,7 +32,8 @@ class MoeBank(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("group", ctypes.c_int32), ("n_exp", ctypes.c_int32),
                 ("reserved", ctypes.c_int32),
                 ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
-                ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p)]
+                ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
+                ("g_gate", ctypes.c_void_p), ("g_up", ctypes.c_void_p), ("g_down", ctypes.c_void_p)]
 
 
 class MoeLayer(ctypes.Structure):
@@ -46,7 +47,8 @@ _LIB = None
 EXPORTS = ["moe_abi_version", "moe_status_str", "moe_validate", "moe_workspace_size",
            "moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
            "moe_layer_forward_marked", "moe_device_status", "moe_launches_per_call",
-           "moe_layer_forward_static", "moe_static_device_status", "moe_test_inject_hold"]
+           "moe_layer_forward_static", "moe_static_device_status", "moe_test_inject_hold",
+           "moe_nvfp4_pack_scales", "moe_nvfp4_quantize_rows"]
 
 
 def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
@@ -80,6 +82,8 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "moe_layer_forward_static": (I32, [LP, P, P, P]),
         "moe_static_device_status": (I32, [ctypes.POINTER(I32), P]),
         "moe_test_inject_hold": (I32, [LP, P, SZ, I32, I32, P]),
+        "moe_nvfp4_pack_scales": (I32, [P, P, I32, I32, I32, P]),
+        "moe_nvfp4_quantize_rows": (I32, [P, I32, I32, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -129,6 +133,11 @@ class DeviceLayer:
                 continue
             self.banks[name] = dict(fmt=bank.fmt, group=bank.group, n_exp=bank.n_exp,
                                     **{k: up(v) for k, v in bank.arrays().items()})
+            if bank.fmt == "nvfp4":  # block scales into the layout the kernels read
+                b = self.banks[name]
+                for m, (N, K) in (("gate", (cfg.f, cfg.d)), ("up", (cfg.f, cfg.d)),
+                                  ("down", (cfg.d, cfg.f))):
+                    b["s_" + m] = nvfp4_pack_scales(b["s_" + m], bank.n_exp, N, K)
 
     @classmethod
     def from_tensors(cls, cfg, router_w, router_bias, routed: dict, shared: dict | None,
@@ -143,10 +152,11 @@ class DeviceLayer:
 
     def _bank(self, b) -> MoeBank:
         if b is None:
-            return MoeBank(16, 128, 0, 0, None, None, None, None, None, None)
+            return MoeBank(16, 128, 0, 0, None, None, None, None, None, None, None, None, None)
         return MoeBank(FMT_CODE[b["fmt"]], b["group"], b["n_exp"], 0,
                        _ptr(b["w_gate"]), _ptr(b["w_up"]), _ptr(b["w_down"]),
-                       _ptr(b.get("s_gate")), _ptr(b.get("s_up")), _ptr(b.get("s_down")))
+                       _ptr(b.get("s_gate")), _ptr(b.get("s_up")), _ptr(b.get("s_down")),
+                       _ptr(b.get("g_gate")), _ptr(b.get("g_up")), _ptr(b.get("g_down")))
 
     def descriptor(self, T: int, path: str | None = None) -> MoeLayer:
         return MoeLayer(T, self.d, self.f, self.E, self.k,
@@ -240,6 +250,32 @@ def layer_forward(L: MoeLayer, x, ws, out=None, topk_idx=None, topk_w=None, offs
                                           _stream(stream), arr, len(marks))
     _check(st, "moe_layer_forward")
     return out
+
+
+def nvfp4_pack_scales(src, n_mats: int, rows: int, K: int, stream=None):
+    """Block scales of an NVFP4 bank, uint8 [n_mats][rows][K/16] on the device, rearranged
+    into the layout the FP4 tensor-core kernels read (a new tensor of the same size)."""
+    import torch
+    src = src.contiguous()
+    dst = torch.empty_like(src)
+    _check(load_library().moe_nvfp4_pack_scales(src.data_ptr(), dst.data_ptr(), n_mats, rows, K,
+                                                _stream(stream)), "moe_nvfp4_pack_scales")
+    return dst
+
+
+def nvfp4_quantize_rows(v, stream=None):
+    """fp32 rows [R, K] on the device -> (E2M1 codes uint8 [R, K/2], E4M3 block-scale codes
+    uint8 [R, K/16], fp32 row scales [R]) by the layer's activation quantiser."""
+    import torch
+    v = v.contiguous()
+    R, K = v.shape
+    codes = torch.empty((R, K // 2), dtype=torch.uint8, device=v.device)
+    scales = torch.empty((R, K // 16), dtype=torch.uint8, device=v.device)
+    g = torch.empty(R, dtype=torch.float32, device=v.device)
+    _check(load_library().moe_nvfp4_quantize_rows(v.data_ptr(), R, K, codes.data_ptr(),
+                                                  scales.data_ptr(), g.data_ptr(),
+                                                  _stream(stream)), "moe_nvfp4_quantize_rows")
+    return codes, scales, g
 
 
 def launches_per_call(L: MoeLayer) -> int:

@@ -126,9 +126,10 @@ __device__ __forceinline__ float warp_topk_gate(uint32_t my_key, uint32_t top_ke
 
 // Everything a kernel needs about one call, resolved on the host.
 struct Bank {
-  int fmt;            // 16, 8, 4
+  int fmt;            // 16, 8, 4, MOE_W_NVFP4
   const void* w[3];   // gate, up, down
-  const uint16_t* s[3];
+  const uint16_t* s[3];  // group scales (NVFP4: the packed E4M3 block scales, as bytes)
+  const float* g[3];     // NVFP4 tensor scales [n_exp] per matrix
 };
 
 struct Plan {
@@ -162,18 +163,29 @@ struct Plan {
   uint16_t* xg;        // tensor-core path: fp16 x rows in grouped order, then the shared
                        // expert's rows [(T*k + T)][d]
   int32_t* tc_sched;   // tensor-core path: per-slot schedule (TcSched view)
+  // NVFP4 routed experts: the activations quantised per grouped row (E2M1 codes, packed
+  // block scales by token tile, fp32 row scales), and h in fp32 before its quantisation
+  uint8_t* xq;         // [T*k][d/2]
+  uint8_t* xsf;        // [token tiles][d/64][512]
+  float* gx;           // [T*k]
+  float* h32;          // [T*k][f]
+  uint8_t* hq;         // [T*k][f/2]
+  uint8_t* hsf;        // [token tiles][f/64][512]
+  float* gh;           // [T*k]
   int path;            // moe_path
 };
 
 // Per slot (active routed experts in ascending order, then the shared expert): rows, first
-// row, expert id (-1: shared) and the running count of 128-row m-tiles, written by
-// tc_prep_kernel. A GEMM with n_tiles weight tiles per expert has units
-// [mt_prefix[s] * n_tiles, mt_prefix[s + 1] * n_tiles) in slot s.
+// row, expert id (-1: shared) and the running count of token tiles (m-tiles of kTcNMax
+// rows), written by tc_prep_kernel. A GEMM with n_tiles weight tiles per expert has units
+// [mt_prefix[s] * n_tiles, mt_prefix[s + 1] * n_tiles) in slot s. expert_mt[e] is the
+// mt_prefix of routed expert e's slot (defined for experts with rows).
 struct TcSched {
   int32_t* slot_rows;    // [E + 2]
   int32_t* slot_row0;    // [E + 2]
   int32_t* slot_expert;  // [E + 2]
   int32_t* mt_prefix;    // [E + 2]; mt_prefix[n_slots] = total m-tiles
+  int32_t* expert_mt;    // [E + 2]
 };
 
 // The synchronisation block at the start of the workspace: status word (offset 0), routing
@@ -204,10 +216,27 @@ cudaError_t launch_tma_down(const Plan& p, cudaStream_t st, bool pdl);
 bool tc_supported(const Plan& p);
 size_t tc_sched_bytes(int E);
 TcSched tc_sched_view(void* base, int E);
-cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st);
+cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st,
+                           bool shared_rows_only = false);
 cudaError_t launch_tc_gate_up(const Plan& p, const TcSched& S, const uint16_t* xg,
                               cudaStream_t st);
 cudaError_t launch_tc_down(const Plan& p, const TcSched& S, cudaStream_t st);
+// the shared expert alone (its bank's format), beside routed experts of another kind
+cudaError_t launch_tc_shared_gate_up(const Plan& p, const TcSched& S, const uint16_t* xg,
+                                     cudaStream_t st);
+cudaError_t launch_tc_shared_down(const Plan& p, const TcSched& S, cudaStream_t st);
+// NVFP4 routed experts on the FP4 tensor cores (nvfp4_grouped.cu)
+constexpr int kNvfp4 = MOE_W_NVFP4;
+size_t nv_tile_cap(int T, int k, int E);  // token tiles a call can have
+bool nv_supported(const Plan& p);
+cudaError_t launch_nv_quant_x(const Plan& p, const TcSched& S, cudaStream_t st);
+cudaError_t launch_nv_gate_up(const Plan& p, const TcSched& S, cudaStream_t st);
+cudaError_t launch_nv_quant_h(const Plan& p, const TcSched& S, cudaStream_t st);
+cudaError_t launch_nv_down(const Plan& p, const TcSched& S, cudaStream_t st);
+cudaError_t launch_nv_quant_rows(const float* v, int rows, int K, uint8_t* codes, uint8_t* scales,
+                                 float* g, cudaStream_t st);
+cudaError_t launch_nv_pack_scales(const uint8_t* src, uint8_t* dst, int n_mats, int rows, int K,
+                                  cudaStream_t st);
 // the whole layer of a 1-token call in one persistent kernel (decode_fused.cu)
 bool decode_fused_supported(const Plan& p);
 cudaError_t launch_decode_fused(const Plan& p, void* out, cudaStream_t st);

@@ -18,11 +18,23 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 bool bank_ok(const moe_bank& b, int expect_n, int d, int f) {
   if (b.n_exp != expect_n) return false;
   if (expect_n == 0) return true;
-  if (b.fmt != MOE_W_BF16 && b.fmt != MOE_W_INT8 && b.fmt != MOE_W_INT4) return false;
+  if (b.fmt != MOE_W_BF16 && b.fmt != MOE_W_INT8 && b.fmt != MOE_W_INT4 && b.fmt != MOE_W_NVFP4)
+    return false;
   const void* w[3] = {b.w_gate, b.w_up, b.w_down};
   for (const void* p : w)
     if (!p || !aligned(p, 16)) return false;
   if (b.fmt == MOE_W_BF16) return true;
+  if (b.fmt == MOE_W_NVFP4) {
+    // packed block scales (bulk copies: 16-byte aligned) and the tensor scales
+    if (b.group != 16) return false;
+    const void* s[3] = {b.s_gate, b.s_up, b.s_down};
+    for (const void* p : s)
+      if (!p || !aligned(p, 16)) return false;
+    const float* g[3] = {b.g_gate, b.g_up, b.g_down};
+    for (const float* p : g)
+      if (!p || !aligned(p, 4)) return false;
+    return true;
+  }
   if (b.group != kGroup) return false;
   const void* s[3] = {b.s_gate, b.s_up, b.s_down};
   for (const void* p : s)
@@ -45,13 +57,21 @@ moe_status validate(const moe_layer* L) {
   if (!bank_ok(L->routed, L->E, L->d, L->f)) return MOE_ERR_INVALID_ARG;
   if (L->shared.n_exp != 0 && L->shared.n_exp != 1) return MOE_ERR_UNSUPPORTED;
   if (!bank_ok(L->shared, L->shared.n_exp, L->d, L->f)) return MOE_ERR_INVALID_ARG;
+  if (L->shared.n_exp && L->shared.fmt == MOE_W_NVFP4) return MOE_ERR_UNSUPPORTED;
+  if (L->routed.fmt == MOE_W_NVFP4) {
+    // the FP4 tensor-core kernels only; stages of 256 K values
+    if (L->path == MOE_PATH_GEMV || L->path == MOE_PATH_FUSED) return MOE_ERR_UNSUPPORTED;
+    if (L->d % 256 || L->f % 256) return MOE_ERR_UNSUPPORTED;
+  }
   return MOE_OK;
 }
+
+inline bool is_nvfp4(const moe_layer* L) { return L->routed.fmt == MOE_W_NVFP4; }
 
 // Workspace layout (offsets from the 256-byte aligned base).
 struct WsLayout {
   size_t status, logits, topk_idx, topk_w, offsets, perm, inv, active, cta_hist, h, y_assign,
-      y_shared, xg, tc_sched, total;
+      y_shared, xg, tc_sched, xq, xsf, gx, h32, hq, hsf, gh, total;
 };
 
 WsLayout layout(const moe_layer* L) {
@@ -74,6 +94,16 @@ WsLayout layout(const moe_layer* L) {
   w.y_shared = take(T * d * sizeof(float));
   w.xg = take((n + T) * d * sizeof(uint16_t));
   w.tc_sched = take(tc_sched_bytes(L->E));
+  // NVFP4 routed experts: quantised activations, block scales by token tile, fp32 h
+  const bool nv = is_nvfp4(L);
+  const size_t tiles = nv ? nv_tile_cap(L->T, L->k, L->E) : 0;
+  w.xq = take(nv ? n * d / 2 : 0);
+  w.xsf = take(tiles * (d / 64) * 512);
+  w.gx = take(nv ? n * sizeof(float) : 0);
+  w.h32 = take(nv ? n * f * sizeof(float) : 0);
+  w.hq = take(nv ? n * f / 2 : 0);
+  w.hsf = take(tiles * (f / 64) * 512);
+  w.gh = take(nv ? n * sizeof(float) : 0);
   w.total = o;
   return w;
 }
@@ -88,6 +118,9 @@ Bank to_bank(const moe_bank& b) {
   r.s[1] = static_cast<const uint16_t*>(b.s_up);
   r.s[2] = static_cast<const uint16_t*>(b.s_down);
   if (b.fmt == MOE_W_BF16) r.s[0] = r.s[1] = r.s[2] = nullptr;
+  r.g[0] = b.fmt == MOE_W_NVFP4 ? b.g_gate : nullptr;
+  r.g[1] = b.fmt == MOE_W_NVFP4 ? b.g_up : nullptr;
+  r.g[2] = b.fmt == MOE_W_NVFP4 ? b.g_down : nullptr;
   return r;
 }
 
@@ -129,6 +162,15 @@ Plan make_plan(const moe_layer* L, void* ws) {
   p.y_shared = reinterpret_cast<float*>(b + w.y_shared);
   p.xg = reinterpret_cast<uint16_t*>(b + w.xg);
   p.tc_sched = reinterpret_cast<int32_t*>(b + w.tc_sched);
+  if (is_nvfp4(L)) {
+    p.xq = b + w.xq;
+    p.xsf = b + w.xsf;
+    p.gx = reinterpret_cast<float*>(b + w.gx);
+    p.h32 = reinterpret_cast<float*>(b + w.h32);
+    p.hq = b + w.hq;
+    p.hsf = b + w.hsf;
+    p.gh = reinterpret_cast<float*>(b + w.gh);
+  }
   p.path = L->path;
   return p;
 }
@@ -174,7 +216,26 @@ bool use_fused(const Plan& p) {
   return decode_fused_supported(p);
 }
 
+// NVFP4 routed experts: the FP4 tensor-core kernels for them, the shared expert (another
+// format) on the integer/bf16 tensor-core kernels.
+moe_status run_ffn_nvfp4(const Plan& p, cudaStream_t st, void* const* marks, int n_marks) {
+  if (!nv_supported(p) || !tc_supported(p)) return MOE_ERR_UNSUPPORTED;
+  if (p.has_shared && !scales_aligned16(p.shared)) return MOE_ERR_UNSUPPORTED;
+  const TcSched S = tc_sched_view(p.tc_sched, p.E);
+  MOE_TRY(launch_tc_prep(p, S, p.xg, st, /*shared_rows_only=*/true));
+  MOE_TRY(launch_nv_quant_x(p, S, st));
+  MOE_TRY(launch_nv_gate_up(p, S, st));
+  if (p.has_shared) MOE_TRY(launch_tc_shared_gate_up(p, S, p.xg, st));
+  MOE_TRY(record_mark(marks, n_marks, 3, st));
+  MOE_TRY(launch_nv_quant_h(p, S, st));
+  MOE_TRY(launch_nv_down(p, S, st));
+  if (p.has_shared) MOE_TRY(launch_tc_shared_down(p, S, st));
+  MOE_TRY(record_mark(marks, n_marks, 4, st));
+  return MOE_OK;
+}
+
 moe_status run_ffn(const Plan& p, cudaStream_t st, void* const* marks, int n_marks) {
+  if (p.routed.fmt == kNvfp4) return run_ffn_nvfp4(p, st, marks, n_marks);
   if (use_tc(p)) {
     if (!tc_supported(p) || !scales_aligned16(p.routed) ||
         (p.has_shared && !scales_aligned16(p.shared)))
@@ -382,6 +443,8 @@ int32_t moe_launches_per_call(const moe_layer* L) {
   }
   if (use_fused(p)) return 1;
   const int route = route_fused_supported(p) ? 1 : (2 + (L->T * L->k <= 1024 ? 1 : 3));
+  if (L->routed.fmt == MOE_W_NVFP4)  // prep, quantise x, gate/up, quantise h, down (+ shared)
+    return route + 5 + (p.has_shared ? 2 : 0) + 1;
   int ffn = use_tc(p) ? 3 : 2;  // (+ gather/schedule) gate/up, down
   if (p.has_shared && p.shared.fmt != p.routed.fmt) ffn += 2;  // each GEMM once per bank
   return route + ffn + 1;       // + combine
@@ -398,6 +461,31 @@ moe_status moe_test_inject_hold(const moe_layer* L, void* ws, size_t ws_bytes, i
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // pageable source: the call returns once the words are staged, so a stack array is fine
   MOE_TRY(cudaMemcpyAsync(dev, words, sizeof(words), cudaMemcpyHostToDevice, st));
+  return MOE_OK;
+}
+
+moe_status moe_nvfp4_pack_scales(const void* src, void* dst, int32_t n_mats, int32_t rows,
+                                 int32_t K, moe_stream_t stream) {
+  if (!src || !dst || !aligned(src, 16) || !aligned(dst, 16)) return MOE_ERR_INVALID_ARG;
+  if (n_mats < 1 || rows < 128 || rows % 128 || K < 64 || K % 64) return MOE_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)n_mats * rows * (K / 16);
+  const uint8_t* a = static_cast<const uint8_t*>(src);
+  const uint8_t* b = static_cast<const uint8_t*>(dst);
+  if (a < b + bytes && b < a + bytes) return MOE_ERR_INVALID_ARG;  // overlap
+  MOE_TRY(launch_nv_pack_scales(a, static_cast<uint8_t*>(dst), n_mats, rows, K,
+                                reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_nvfp4_quantize_rows(const float* v, int32_t rows, int32_t K, void* codes,
+                                   void* scales, float* g, moe_stream_t stream) {
+  if (!v || !codes || !scales || !g) return MOE_ERR_INVALID_ARG;
+  if (!aligned(v, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(g, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (rows < 1 || K < 16 || K % 16 || K > 8192) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(launch_nv_quant_rows(v, rows, K, static_cast<uint8_t*>(codes),
+                               static_cast<uint8_t*>(scales), g,
+                               reinterpret_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 

@@ -43,10 +43,9 @@
 
 #include <cuda_fp16.h>
 
-#include "pipeline.cuh"
+#include "tc_common.cuh"
 
 namespace moe {
-
 
 constexpr int kTcThreads = 512;  // 16 warps
 constexpr int kDqWarps = 8;       // dequantisers (two threads per weight row)
@@ -54,9 +53,6 @@ constexpr int kIssuers = 2;       // MMA issuing warps (1 and 14)
 // threads of one chunk's ready barrier: a dequantiser group of four warps and the issuers
 constexpr int kReadyThreads = 32 * (kDqWarps / 2 + kIssuers);
 constexpr int kTcBK = 64;      // K per chunk (one 128-byte swizzle span of bf16)
-constexpr int kTcM = 128;      // weight rows per tile
-constexpr int kTcNMax = 64;    // token rows per tile
-constexpr int kBoxes = 3;      // activation boxes of 16, 32, 64 rows
 
 struct TcMaps {
   CUtensorMap w[2][2];          // [bank: routed, shared][matrix: gate|down, up]
@@ -118,36 +114,6 @@ __host__ __device__ inline TcSmem tc_smem(int K, int E) {
   return m;
 }
 
-// ------------------------------------------------------------------ PTX wrappers
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
 
 // Warp-level forms: the whole (converged) warp executes them and one elected lane issues.
 // Issuing from a converged warp costs a fraction of issuing from a lone lane of a diverged
@@ -162,15 +128,6 @@ __device__ __forceinline__ void umma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tme
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-
-__device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
 // 32 consecutive 32-bit columns of this thread's TMEM lane <- registers (one wide
 // instruction: every tcgen05 instruction has a sizeable fixed issue cost).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -188,69 +145,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-
-// 16 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// UMMA shared-memory descriptor, K-major, 128-byte swizzle: rows of 128 bytes, groups of
-// 8 rows 1024 bytes apart (SBO), version 1 (sm_100), layout type 2 (128B swizzle).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-  d |= (uint64_t)1 << 16;                 // LBO (unused for swizzled K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;       // SBO
-  d |= (uint64_t)1 << 46;                 // version
-  d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
-  return d;
-}
-
 // Instruction descriptor: D fp32, A and B fp16, both K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t umma_idesc_f16(int n) {
   return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTcM >> 4) << 24);
-}
-
-// ------------------------------------------------------------------ schedule
-
-struct TcUnit {
-  int slot, e, shared, row0, nrows, ntile, mtile;
-};
-
-// S points at the CTA's shared-memory copy of the schedule.
-__device__ __forceinline__ TcUnit tc_unit(const TcSched& S, int n_slots, int n_tiles, int u) {
-  int lo = 0, hi = n_slots;  // largest s with mt_prefix[s] * n_tiles <= u
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (S.mt_prefix[mid] * n_tiles <= u) lo = mid;
-    else hi = mid;
-  }
-  TcUnit t;
-  t.slot = lo;
-  const int local = u - S.mt_prefix[lo] * n_tiles;
-  const int mts = (S.slot_rows[lo] + kTcNMax - 1) / kTcNMax;
-  t.ntile = local / mts;
-  t.mtile = local % mts;
-  t.e = S.slot_expert[lo];
-  t.shared = (t.e < 0);
-  if (t.shared) t.e = 0;
-  t.row0 = S.slot_row0[lo] + t.mtile * kTcNMax;
-  t.nrows = min(kTcNMax, S.slot_rows[lo] - t.mtile * kTcNMax);
-  return t;
-}
-
-__device__ __forceinline__ int box_index(int nrows) {
-  return nrows <= 16 ? 0 : (nrows <= 32 ? 1 : (nrows <= 64 ? 2 : 3));
 }
 
 // K order of the fp16 operands the tensor core reads. For int4 weights the dequantisers
@@ -267,8 +164,10 @@ __device__ __forceinline__ int k_position(int n, bool interleave) {
 }
 
 // Gathers the activation rows in fp16 (xg[r] = x[perm[r] / k] for the T*k grouped rows, then
-// xg[T*k + t] = x[t] for the shared expert) and, in CTA 0, builds the unit schedule.
-__global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_t* xg) {
+// xg[T*k + t] = x[t] for the shared expert; rows from row_begin on) and, in CTA 0, builds the
+// unit schedule.
+__global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_t* xg,
+                                                      int row_begin) {
   pdl_wait();
   if (blockIdx.x == 0) {
     __shared__ int s_units[kMaxE + 1];
@@ -295,6 +194,7 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
       int run = 0;
       for (int s = 0; s < n_slots; ++s) {
         S.mt_prefix[s] = run;
+        if (s < n_active) S.expert_mt[S.slot_expert[s]] = run;
         run += s_units[s];
       }
       S.mt_prefix[n_slots] = run;
@@ -308,7 +208,8 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
     const int chunks = p.d / 8;
     const int warps = blockDim.x / 32, lane = threadIdx.x & 31;
     bool range_ok = true;
-    for (int r = blockIdx.x * warps + (int)(threadIdx.x >> 5); r < rows; r += gridDim.x * warps) {
+    for (int r = row_begin + blockIdx.x * warps + (int)(threadIdx.x >> 5); r < rows;
+         r += gridDim.x * warps) {
       const int t = (r < n) ? p.perm[r] / p.k : r - n;
       const bool il = interleaved_k((r < n) ? p.routed.fmt : p.shared.fmt);
       const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)t * p.d);
@@ -791,39 +692,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void* ptr = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// 2-D map over a row-major [rows][cols] array.
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t cols,
-              uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
-  auto enc = get_encoder();
-  if (!enc || !base) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * esize};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
-size_t tc_sched_bytes(int E) { return sizeof(int32_t) * (size_t)(4 * (E + 2)); }
+size_t tc_sched_bytes(int E) { return sizeof(int32_t) * (size_t)(5 * (E + 2)); }
 
 TcSched tc_sched_view(void* base, int E) {
   int32_t* b = static_cast<int32_t*>(base);
@@ -832,6 +702,7 @@ TcSched tc_sched_view(void* base, int E) {
   s.slot_row0 = b + (E + 2);
   s.slot_expert = b + 2 * (E + 2);
   s.mt_prefix = b + 3 * (E + 2);
+  s.expert_mt = b + 4 * (E + 2);
   return s;
 }
 
@@ -936,8 +807,10 @@ bool tc_supported(const Plan& p) {
          p.d % kTcBK == 0 && p.f % kTcBK == 0;
 }
 
-cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st) {
-  const long long rows = (long long)p.T * p.k + p.T;  // one warp a row, 8 rows a CTA
+cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaStream_t st,
+                           bool shared_rows_only) {
+  const int row_begin = shared_rows_only ? p.T * p.k : 0;
+  const long long rows = (long long)p.T * p.k + p.T - row_begin;  // one warp a row, 8 a CTA
   const int blocks = (int)std::max(1LL, std::min<long long>(1184, (rows + 7) / 8));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
@@ -948,7 +821,7 @@ cudaError_t launch_tc_prep(const Plan& p, const TcSched& S, uint16_t* xg, cudaSt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_prep_kernel, p, S, xg);
+  return cudaLaunchKernelEx(&cfg, tc_prep_kernel, p, S, xg, row_begin);
 }
 
 // Gate/up with two accumulator buffers when the routed experts average 32 rows or more.
@@ -959,6 +832,14 @@ cudaError_t launch_tc_gate_up(const Plan& p, const TcSched& S, const uint16_t* x
 }
 cudaError_t launch_tc_down(const Plan& p, const TcSched& S, cudaStream_t st) {
   return launch_tc<false, 2>(p, S, nullptr, st);
+}
+
+cudaError_t launch_tc_shared_gate_up(const Plan& p, const TcSched& S, const uint16_t* xg,
+                                     cudaStream_t st) {
+  return launch_tc_part<true, 1>(p, S, xg, p.shared.fmt, 2, st);
+}
+cudaError_t launch_tc_shared_down(const Plan& p, const TcSched& S, cudaStream_t st) {
+  return launch_tc_part<false, 2>(p, S, nullptr, p.shared.fmt, 2, st);
 }
 
 }  // namespace moe

@@ -147,10 +147,14 @@ def e2m1_codes(v: np.ndarray) -> np.ndarray:
     """float32 values -> E2M1 codes (uint8), nearest, ties to the even code, saturating."""
     a = np.abs(v).astype(np.float32)
     mids = (_E2M1_GRID[1:] + _E2M1_GRID[:-1]) / np.float32(2)
-    i = np.searchsorted(mids, a, side="left")  # mids strictly below a
-    tie = (i < len(mids)) & (a == mids[np.minimum(i, len(mids) - 1)])
-    i = np.where(tie & (i % 2 == 1), i + 1, i)
-    return (i.astype(np.uint8) | (np.signbit(v).astype(np.uint8) << 3)).astype(np.uint8)
+    i = np.zeros(a.shape, np.uint8)  # number of mids strictly below a
+    tie = np.zeros(a.shape, bool)    # a on a mid whose lower neighbour has an odd code
+    for m, mid in enumerate(mids):
+        i += a > mid
+        if m % 2 == 1:
+            tie |= a == mid
+    i += tie
+    return i | (np.signbit(v).astype(np.uint8) << 3)
 
 
 def e4m3_codes(v: np.ndarray) -> np.ndarray:
@@ -284,11 +288,21 @@ def _make_nvfp4_bank(cfg: LayerConfig, which: str, n_exp: int, experts=None) -> 
                       np.zeros((n_exp, N, K // NVFP4_BLOCK), np.uint8),
                       np.zeros(n_exp, np.float32))
     todo = range(n_exp) if experts is None else experts
-    for e in todo:
-        for name, (N, K) in (("gate", (f, d)), ("up", (f, d)), ("down", (d, f))):
-            w = _normal((N, K), cfg.weight_std, cfg.seed, which, name, int(e))
-            q, sc, g = quantize_nvfp4(w)
-            arrs[name][0][e], arrs[name][1][e], arrs[name][2][e] = q, sc, g
+    jobs = [(int(e), name, N, K) for e in todo
+            for name, (N, K) in (("gate", (f, d)), ("up", (f, d)), ("down", (d, f)))]
+
+    def one(job):
+        e, name, N, K = job
+        w = _normal((N, K), cfg.weight_std, cfg.seed, which, name, e)
+        q, sc, g = quantize_nvfp4(w)
+        arrs[name][0][e], arrs[name][1][e], arrs[name][2][e] = q, sc, g
+
+    if len(jobs) <= 3:
+        for j in jobs:
+            one(j)
+    else:
+        with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+            list(ex.map(one, jobs))
     return Bank("nvfp4", NVFP4_BLOCK, n_exp, d, f, arrs["gate"][0], arrs["up"][0], arrs["down"][0],
                 arrs["gate"][1], arrs["up"][1], arrs["down"][1],
                 arrs["gate"][2], arrs["up"][2], arrs["down"][2])

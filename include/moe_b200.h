@@ -35,6 +35,20 @@
  *                   S[e][n][k / group].
  *       MOE_W_INT4  W[e][n][k / 8] uint32, 8 two's-complement nibbles per word along K,
  *                   element k at bits 4 * (k % 8) of word k / 8; scales as for int8.
+ *       MOE_W_NVFP4 (routed bank only) NVFP4, the W4A4 variant of the layer (Anvil serving
+ *                   benchmarks, "Qwen3.8 Flash Next", "Quantization boundary": ModelOpt
+ *                   NVFP4 W4A4 on the routed experts, the shared expert kept BF16):
+ *                   W[e][n][k / 2] uint8 of E2M1 codes, element k at bits 4 * (k % 2) of
+ *                   byte k / 2; one E4M3 scale per 16 consecutive K values, stored in the
+ *                   tensor-core layout that moe_nvfp4_pack_scales writes (group = 16);
+ *                   one fp32 tensor scale per expert matrix in g_gate / g_up / g_down
+ *                   ([n_exp] each). value = e2m1 * e4m3 * g. The activations entering the
+ *                   routed experts (x, and h = silu(gate) * up rounded to fp32) are
+ *                   quantised to NVFP4 per row at run time: g_row = amax / (6 * 448),
+ *                   block scale = E4M3(amax_block / (6 g_row)), element =
+ *                   E2M1(v / (block scale * g_row)), both nearest-even, every step an
+ *                   IEEE fp32 operation. Such layers run on the FP4 tensor cores
+ *                   (tcgen05.mma kind::mxf4nvf4) for every T; path must be AUTO or TC.
  *     gate and up are [n_exp][f][d] (N = f, K = d); down is [n_exp][d][f] (N = d, K = f).
  *     The two banks may use different encodings (e.g. an int8 shared expert beside int4
  *     routed experts); the grouped products then run once per bank. The single-kernel
@@ -53,7 +67,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -74,7 +88,7 @@ typedef enum {
   MOE_ERR_TOO_LARGE = -7    /* the request needs more than the library's built-in scratch */
 } moe_status;
 
-typedef enum { MOE_W_BF16 = 16, MOE_W_INT8 = 8, MOE_W_INT4 = 4 } moe_wfmt;
+typedef enum { MOE_W_BF16 = 16, MOE_W_INT8 = 8, MOE_W_INT4 = 4, MOE_W_NVFP4 = 41 } moe_wfmt;
 
 /* Which kernels run. AUTO picks the single-kernel layer (FUSED) for 1-token calls with
  * int4 banks when the device fits it, the split-K GEMV kernels for other calls of 1..15
@@ -89,15 +103,18 @@ typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC = 2, MOE_PATH_F
  * slice starts at e * (N * K * bits / 8) bytes. */
 typedef struct {
   int32_t fmt;   /* moe_wfmt */
-  int32_t group; /* 128 for MOE_W_INT8 / MOE_W_INT4; ignored for MOE_W_BF16 */
+  int32_t group; /* 128 for MOE_W_INT8 / MOE_W_INT4, 16 for MOE_W_NVFP4; ignored for bf16 */
   int32_t n_exp;
   int32_t reserved;
   const void* w_gate; /* [n_exp][f][d] encoded */
   const void* w_up;   /* [n_exp][f][d] encoded */
   const void* w_down; /* [n_exp][d][f] encoded */
-  const void* s_gate; /* bf16 [n_exp][f][d / group] or NULL (bf16 weights) */
-  const void* s_up;   /* bf16 [n_exp][f][d / group] or NULL */
-  const void* s_down; /* bf16 [n_exp][d][f / group] or NULL */
+  const void* s_gate; /* bf16 [n_exp][f][d / group], packed E4M3 (NVFP4), or NULL (bf16) */
+  const void* s_up;   /* bf16 [n_exp][f][d / group], packed E4M3 (NVFP4), or NULL */
+  const void* s_down; /* bf16 [n_exp][d][f / group], packed E4M3 (NVFP4), or NULL */
+  const float* g_gate; /* NVFP4 only: fp32 [n_exp] tensor scales (NULL otherwise) */
+  const float* g_up;
+  const float* g_down;
 } moe_bank;
 
 /* The layer: shapes, router and the two banks. Read by every call; not retained. */
@@ -228,6 +245,29 @@ MOE_API moe_status moe_layer_forward_static(const moe_layer* L, const void* x, v
  * of any call since the last read is reported here. Allocates nothing. Like the first static
  * call, the first call of this function on a device looks up the buffer's address. */
 MOE_API moe_status moe_static_device_status(int32_t* code, moe_stream_t stream);
+
+/* Block scales of an NVFP4 bank in the layout its kernels read. `src` holds one E4M3 byte per
+ * 16 consecutive K values of each row, row-major: uint8 [n_mats][rows][K / 16] (the natural
+ * order). `dst` (same size, caller-owned, 16-byte aligned) receives, for each matrix, each
+ * tile of 128 rows and each step of 64 K values, one 512-byte block in which the scale of row
+ * 128 * tile + 32 * q + i (i < 32, q < 4) for K values 64 * step + 16 * j .. +15 (j < 4) sits at
+ * byte 16 * i + 4 * q + j: the order in which the tensor core takes a 128-row operand's scales
+ * into tensor memory (tcgen05.cp, 32 lanes x 128 bits, repeated in the four lane quarters).
+ * Call once per bank when the weights are loaded; pass dst as the bank's s_* pointer.
+ * rows % 128 == 0, K % 64 == 0, n_mats >= 1. Enqueued on `stream`; src and dst must not
+ * overlap. Returns MOE_ERR_INVALID_ARG for a bad size or pointer. */
+MOE_API moe_status moe_nvfp4_pack_scales(const void* src, void* dst, int32_t n_mats, int32_t rows,
+                                         int32_t K, moe_stream_t stream);
+
+/* NVFP4 quantisation of fp32 rows, as the layer applies it to the activations entering NVFP4
+ * routed experts: per row, g = amax / (6 * 448) (fp32 [rows]); per block of 16 values the E4M3
+ * code of amax_block / (6 g), nearest even, saturating at 448 (uint8 [rows][K / 16], natural
+ * order); the E2M1 codes of v / (e4m3 * g), nearest even, saturating at 6 (uint8
+ * [rows][K / 2], element k at bits 4 * (k % 2) of byte k / 2); each step one IEEE fp32
+ * operation; a zero row gives zero codes. v: fp32 [rows][K], K % 16 == 0, K <= 8192, rows >= 1;
+ * every pointer 16-byte aligned (g: 4). Enqueued on `stream`. */
+MOE_API moe_status moe_nvfp4_quantize_rows(const float* v, int32_t rows, int32_t K, void* codes,
+                                           void* scales, float* g, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

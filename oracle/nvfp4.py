@@ -139,11 +139,16 @@ def nvfp4_quantize_rows(v32: np.ndarray):
     return codes, sc, g
 
 
+# every code's value, from the definitions above (a table lookup decodes whole matrices fast)
+_E2M1_TABLE = e2m1_value(np.arange(16))
+_E4M3_TABLE = e4m3_value(np.arange(256))
+
+
 def nvfp4_dequantize(codes: np.ndarray, scale_codes: np.ndarray, g: np.ndarray) -> np.ndarray:
     """E2M1 codes [..., K], E4M3 block-scale codes [..., K/16], float32 tensor scale(s)
     (broadcast over the leading axes) -> float64 values (exact)."""
-    v = e2m1_value(codes)
-    s = np.repeat(e4m3_value(scale_codes), BLOCK, axis=-1)
+    v = _E2M1_TABLE[np.asarray(codes).astype(np.int64) & 0xF]
+    s = np.repeat(_E4M3_TABLE[np.asarray(scale_codes).astype(np.int64) & 0xFF], BLOCK, axis=-1)
     return v * s * np.asarray(g, np.float64)[..., None]
 
 
@@ -171,11 +176,13 @@ def expert_ffn_w4a4(x32: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndar
 
 
 def layer_forward_nvfp4(x_bits, router_w, router_bias, routed: dict, shared: dict | None,
-                        k: int) -> dict:
+                        k: int, tokens=None) -> dict:
     """The layer with NVFP4 W4A4 routed experts (``routed``: dict with fmt "nvfp4", packed
     E2M1 codes w_*, E4M3 block scales s_*, float32 tensor scales g_* per expert) and an
-    optional BF16/int shared expert (``shared``: a bank dict of ``moe_oracle``). Returns the
-    same fields as ``moe_oracle.layer_forward``."""
+    optional BF16/int shared expert (``shared``: a bank dict of ``moe_oracle``). ``tokens``
+    optionally restricts which output rows are computed (routing and the plan always cover
+    all tokens; a row's result depends on that row alone). Returns the same fields as
+    ``moe_oracle.layer_forward`` (``out``: float64 [len(tokens), d])."""
     assert routed["fmt"] == "nvfp4"
     x = M.widen_bf16(x_bits)                      # bf16 values, exact in float32
     T, d = x.shape
@@ -185,28 +192,30 @@ def layer_forward_nvfp4(x_bits, router_w, router_bias, routed: dict, shared: dic
     idx, gates = M.select_topk(logits, k)
     counts, offsets, perm, inv = M.route_plan(idx, E)
     x32 = x.astype(np.float32)
-    # y for every (token, slot), expert by expert (each expert decoded once); a row is
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    pos = {int(t): i for i, t in enumerate(tokens)}
+    # y for every needed (token, slot), expert by expert (each expert decoded once); a row is
     # quantised on its own (N2), so grouping rows does not change any row's result
-    y = np.zeros((T, k, d), np.float64)
+    y = np.zeros((len(tokens), k, d), np.float64)
     needed = {}
-    for t in range(T):
+    for t in tokens:
         for j in range(k):
-            needed.setdefault(int(idx[t, j]), []).append((t, j))
+            needed.setdefault(int(idx[t, j]), []).append((int(t), j))
     for e in sorted(needed):
         Wg, Wu, Wd = _weights(routed, e, d, f)
         rows = needed[e]
         ys = expert_ffn_w4a4(x32[[t for t, _ in rows]], Wg, Wu, Wd)
         for (t, j), yy in zip(rows, ys):
-            y[t, j] = yy
-    out = np.zeros((T, d), np.float64)
-    for t in range(T):
+            y[pos[t], j] = yy
+    out = np.zeros((len(tokens), d), np.float64)
+    for i in range(len(tokens)):
         acc = np.zeros(d, np.float64)
         for j in range(k):                        # rank order, then the shared expert
-            acc = acc + gates[t, j] * y[t, j]
-        out[t] = acc
+            acc = acc + gates[tokens[i], j] * y[i, j]
+        out[i] = acc
     if shared is not None:
         for s in range(shared["w_gate"].shape[0]):
             Wg, Wu, Wd = M._bank_expert(shared, s, d, f)
-            out += M.expert_ffn(x, Wg, Wu, Wd)
+            out += M.expert_ffn(x[tokens], Wg, Wu, Wd)
     return dict(logits=logits, idx=idx, gates=gates, counts=counts, offsets=offsets,
                 perm=perm, inv=inv, out=out)

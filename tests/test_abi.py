@@ -28,7 +28,7 @@ def test_exports_match_header(lib):
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(binding.EXPORTS)
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
 
 
 def _desc(**kw):
@@ -71,6 +71,56 @@ def test_validation_banks(lib):
     d.routed.s_gate = d.routed.s_up = d.routed.s_down = None
     d.shared.fmt = 16
     assert lib.moe_validate(ctypes.byref(d)) == 0
+
+
+def _nvfp4_desc(**kw):
+    fake = 1 << 20
+    d = _desc(**kw)
+    d.routed = binding.MoeBank(41, 16, 512, 0, fake, fake, fake, fake, fake, fake,
+                               fake, fake, fake)
+    d.shared.fmt = 16
+    d.shared.s_gate = d.shared.s_up = d.shared.s_down = None
+    return d
+
+
+def test_validation_nvfp4_bank(lib):
+    d = _nvfp4_desc()
+    assert lib.moe_validate(ctypes.byref(d)) == 0
+    nv_ws = lib.moe_workspace_size(ctypes.byref(d))
+    d.path = binding.PATH_CODE["tc"]
+    assert lib.moe_validate(ctypes.byref(d)) == 0
+    for path in ("gemv", "fused"):  # the FP4 tensor-core kernels only
+        d.path = binding.PATH_CODE[path]
+        assert lib.moe_validate(ctypes.byref(d)) == -2
+    d = _nvfp4_desc()
+    d.routed.group = 128  # NVFP4 blocks are 16 values
+    assert lib.moe_validate(ctypes.byref(d)) == -1
+    d = _nvfp4_desc()
+    d.routed.g_up = None  # tensor scales required
+    assert lib.moe_validate(ctypes.byref(d)) == -1
+    d = _nvfp4_desc()
+    d.routed.s_down = (1 << 20) + 8  # packed scales are read by bulk copies: 16-byte aligned
+    assert lib.moe_validate(ctypes.byref(d)) == -1
+    d = _nvfp4_desc(d=2560 + 128)  # stages of 256 K values
+    assert lib.moe_validate(ctypes.byref(d)) == -2
+    d = _nvfp4_desc()
+    d.shared = binding.MoeBank(41, 16, 1, 0, *([1 << 20] * 9))  # routed experts only
+    assert lib.moe_validate(ctypes.byref(d)) == -2
+    # the NVFP4 intermediates (quantised x and h, fp32 h) add to the integer layer's workspace
+    assert nv_ws > lib.moe_workspace_size(ctypes.byref(_desc()))
+
+
+def test_nvfp4_helpers_validate_on_host(lib):
+    fake = 1 << 20
+    pack = lib.moe_nvfp4_pack_scales
+    assert pack(None, fake, 1, 128, 64, None) == -1
+    assert pack(fake, fake + (1 << 20), 1, 100, 64, None) == -1   # rows % 128
+    assert pack(fake, fake + (1 << 20), 1, 128, 48, None) == -1    # K % 64
+    assert pack(fake, fake + 64, 1, 128, 64, None) == -1           # overlapping buffers
+    q = lib.moe_nvfp4_quantize_rows
+    assert q(fake, 4, 40, fake, fake, fake, None) == -1            # K % 16
+    assert q(fake, 0, 64, fake, fake, fake, None) == -1            # rows
+    assert q(fake + 8, 4, 64, fake, fake, fake, None) == -1        # alignment
 
 
 def test_workspace_size_grows_with_T(lib):
