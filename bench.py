@@ -42,7 +42,9 @@ HBM_NOMINAL_GBS = 8000.0      # the HBM3e figure the decode target is stated aga
 TC_NOMINAL_TFLOPS = 2250.0    # dense bf16/fp16 tensor-core peak of one B200
 L2_BYTES = 126 * 2 ** 20
 POOL = 64
-ALL_WORKLOADS = ("decode", "verify16", "verify32", "prefill", "long")
+ALL_WORKLOADS = ("decode", "verify16", "verify32", "prefill", "long", "prefill_nvfp4",
+                 "long_nvfp4")
+FP4_OVER_BF16 = 4.0           # nominal dense FP4 / BF16 tensor-core ratio of a B200 (9 / 2.25)
 HEADLINE = "decode"
 
 
@@ -72,10 +74,19 @@ def measured_peaks():
     return HBM_FALLBACK_GBS, TC_FALLBACK_TFLOPS, TC_FALLBACK_TFLOPS, "fallback"
 
 
-def bank_bytes_per_expert(cfg):
-    bits = synth.FMT_BITS[cfg.fmt]
+def bank_bytes_per_expert(cfg, fmt=None):
+    """(weight bytes, scale bytes) of one expert (gate, up, down) in ``fmt`` (default: the
+    routed bank's format). NVFP4: 4-bit codes, one E4M3 byte per 16 values, three fp32
+    tensor scales."""
+    fmt = cfg.fmt if fmt is None else fmt
+    bits = synth.FMT_BITS[fmt]
     w = 3 * cfg.d * cfg.f * bits // 8
-    s = 0 if cfg.fmt == "bf16" else 3 * cfg.d * cfg.f // cfg.group * 2
+    if fmt == "bf16":
+        s = 0
+    elif fmt == "nvfp4":
+        s = 3 * cfg.d * cfg.f // 16 + 3 * 4
+    else:
+        s = 3 * cfg.d * cfg.f // cfg.group * 2
     return w, s
 
 
@@ -106,8 +117,11 @@ def replicas_for(cfg, requested=0):
 def workload_config(cfg, world, replicas=0):
     """The ``config`` object of a bench line (identical for both arms)."""
     R = replicas_for(cfg, replicas)
+    weights = (f"{cfg.fmt} g{cfg.group}" if cfg.fmt != "nvfp4" else
+               "nvfp4 routed (E2M1, E4M3 per 16, fp32 per matrix; activations NVFP4 per row), "
+               f"{cfg.shared_fmt or cfg.fmt} shared")
     return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-            "f": cfg.f, "n_shared": cfg.n_shared, "weights": f"{cfg.fmt} g{cfg.group}",
+            "f": cfg.f, "n_shared": cfg.n_shared, "weights": weights,
             "router": "bf16, fp32 logits" + (", Zipf(1.1) bias" if cfg.zipf_s else ""),
             "parallelism": f"replicas x{world}",
             "l2": (f"inputs larger than L2: {R} weight copies x {pool_size(cfg)} hidden "
@@ -130,7 +144,8 @@ def max_over_ranks(values, device="cpu"):
 KERNEL_SOURCES = {
     "decode_fused": ("decode_fused.cu", "gemv_frag.cuh", "pipeline.cuh", "common.cuh"),
     "gemv_tma": ("gemv_tma.cu", "gemv_frag.cuh", "pipeline.cuh", "common.cuh"),
-    "tc_grouped": ("tc_grouped.cu", "pipeline.cuh", "common.cuh"),
+    "tc_grouped": ("tc_grouped.cu", "tc_common.cuh", "pipeline.cuh", "common.cuh"),
+    "nv_grouped": ("nvfp4_grouped.cu", "tc_common.cuh", "pipeline.cuh", "common.cuh"),
 }
 
 
@@ -213,7 +228,8 @@ def _blas_threads():
 # Tokens of the batched oracle call timed per workload: the whole batch where that ends in
 # seconds, else the first tokens of it (the oracle dequantises each touched expert once per
 # call, about 0.1 s an expert, so its cost grows with the experts a slice touches).
-CPU_SLICE = {"tiny": 64, "decode": 1, "verify16": 8, "verify32": 8, "prefill": 16, "long": 64}
+CPU_SLICE = {"tiny": 64, "decode": 1, "verify16": 8, "verify32": 8, "prefill": 16, "long": 64,
+             "prefill_nvfp4": 8, "long_nvfp4": 32}
 
 
 def cpu_oracle_rate(cfg, L, seconds, n_tokens=None):
@@ -222,13 +238,15 @@ def cpu_oracle_rate(cfg, L, seconds, n_tokens=None):
     dequantised once per call, as the workload's own call does), repeated until ``seconds``
     pass (at least one call)."""
     from oracle import moe_oracle as O
+    from oracle import nvfp4 as NV
     routed, shared = _oracle_bank(L.routed), _oracle_bank(L.shared)
+    forward = NV.layer_forward_nvfp4 if cfg.fmt == "nvfp4" else O.layer_forward
     n = L.x.shape[0] if n_tokens is None else min(n_tokens, L.x.shape[0])
     x = L.x[:n]
     t0 = time.perf_counter()
     done = calls = 0
     while True:
-        O.layer_forward(x, L.router_w, L.router_bias, routed, shared, cfg.k)
+        forward(x, L.router_w, L.router_bias, routed, shared, cfg.k)
         done += n
         calls += 1
         if time.perf_counter() - t0 >= seconds:
@@ -358,6 +376,9 @@ def run_workload(name, args, world, local_rank, cache):
 
     w_b, s_b = bank_bytes_per_expert(cfg)
     per_exp = w_b + s_b
+    nv = cfg.fmt == "nvfp4"
+    sw_b, ss_b = bank_bytes_per_expert(cfg, cfg.shared_fmt or cfg.fmt)
+    per_shared = (sw_b + ss_b) if L.shared is not None else 0
     router_b = cfg.E * cfg.d * 2
     R = replicas_for(cfg, args.replicas)
     layers = [base]
@@ -377,12 +398,22 @@ def run_workload(name, args, world, local_rank, cache):
 
     # ---- algorithmic bytes per pool entry: the layer, and its grouped gate/up launch
     gu_bytes, layer_bytes = [], []
+    n_rows = cfg.T * cfg.k
     for xd in x_dev:
         B.layer_forward(descs[0], xd, ws, out=out, topk_idx=idx_buf)
-        u = np.unique(idx_buf.cpu().numpy()).size + (1 if L.shared is not None else 0)
-        gu = u * (2 * per_exp // 3) + cfg.T * cfg.d * 2 + (cfg.T * cfg.k + cfg.T) * cfg.f * 2
+        ur = np.unique(idx_buf.cpu().numpy()).size  # routed experts touched
+        if nv:
+            # gate/up stage: routed gate/up codes and scales, the shared expert's gate/up, x
+            # (bf16, read to quantise), the quantised rows read by the GEMM, h written (fp32)
+            gu = (ur * (2 * per_exp // 3) + 2 * per_shared // 3 + cfg.T * cfg.d * 2
+                  + n_rows * cfg.d * 9 // 16 + n_rows * cfg.f * 4 + cfg.T * cfg.f * 2)
+            lb = ur * per_exp + per_shared + router_b + 2 * cfg.T * cfg.d * 2
+        else:
+            u = ur + (1 if L.shared is not None else 0)
+            gu = u * (2 * per_exp // 3) + cfg.T * cfg.d * 2 + (n_rows + cfg.T) * cfg.f * 2
+            lb = u * per_exp + router_b + 2 * cfg.T * cfg.d * 2
         gu_bytes.append(gu)
-        layer_bytes.append(u * per_exp + router_b + 2 * cfg.T * cfg.d * 2)
+        layer_bytes.append(lb)
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream(device=dev)
@@ -477,8 +508,13 @@ def run_workload(name, args, world, local_rank, cache):
         k_ms_avg = float(np.mean(k_ms))
         achieved = float(np.sum(k_bytes) / (np.sum(k_ms) * 1e-3) / 1e9)
         tc = cfg.T >= 16
-        kernel_name = "grouped gate/up + SwiGLU" + (" (tcgen05, with its row gather)" if tc else "")
-        prof_kernel = "tc_grouped" if tc else "gemv_tma"
+        if nv:
+            kernel_name = ("grouped gate/up + SwiGLU stage (FP4 tcgen05 kind::mxf4nvf4 with the "
+                           "activation quantiser, and the bf16 shared expert)")
+            prof_kernel = "nv_grouped"
+        else:
+            kernel_name = "grouped gate/up + SwiGLU" + (" (tcgen05, with its row gather)" if tc else "")
+            prof_kernel = "tc_grouped" if tc else "gemv_tma"
 
     # ---- end to end through the public call with host buffers
     x_host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -506,6 +542,27 @@ def run_workload(name, args, world, local_rank, cache):
     layer_gbs = lb / (ms_per_step * 1e-3) / 1e9
     flops = layer_flops(cfg)
     tflops = flops / (ms_per_step * 1e-3) / 1e12
+    tensor = {"flops_per_step": flops, "achieved_tflops": tflops,
+              "peak_sustained": tc_sust, "frac": tflops / tc_sust,
+              "peak_burst": tc_burst, "frac_burst": tflops / tc_burst,
+              "peak_nominal": TC_NOMINAL_TFLOPS, "frac_nominal": tflops / TC_NOMINAL_TFLOPS}
+    if nv:
+        # routed experts on the FP4 tensor cores (peak: the measured bf16 figure x the nominal
+        # FP4/BF16 ratio), shared expert and router at the bf16 rate: the fraction is the time
+        # the contraction needs at those peaks over the step time
+        f_routed = 2 * 3 * cfg.d * cfg.f * cfg.T * cfg.k
+        f_rest = flops - f_routed
+
+        def ideal_s(peak_tf):
+            return (f_routed / (FP4_OVER_BF16 * peak_tf) + f_rest / peak_tf) / 1e12
+
+        step_s = ms_per_step * 1e-3
+        tensor.update(frac=ideal_s(tc_sust) / step_s, frac_burst=ideal_s(tc_burst) / step_s,
+                      frac_nominal=ideal_s(TC_NOMINAL_TFLOPS) / step_s,
+                      fp4_flops_per_step=f_routed,
+                      peak_fp4_sustained=FP4_OVER_BF16 * tc_sust,
+                      peak_kind="fp4 = measured bf16 x 4 (nominal ratio) for the routed "
+                                "experts, measured bf16 for the rest")
     roof = {"bound": "hbm", "kernel": kernel_name, "achieved": achieved, "peak": hbm,
             "unit": "GB/s", "frac": achieved / hbm, "peak_kind": peak_kind,
             "frac_nominal": achieved / HBM_NOMINAL_GBS,
@@ -513,11 +570,7 @@ def run_workload(name, args, world, local_rank, cache):
             "avg_launch_ms": k_ms_avg,
             "layer_bytes": lb, "layer_achieved": layer_gbs, "layer_frac": layer_gbs / hbm,
             "layer_frac_nominal": layer_gbs / HBM_NOMINAL_GBS,
-            "tensor": {"flops_per_step": flops, "achieved_tflops": tflops,
-                       "peak_sustained": tc_sust, "frac": tflops / tc_sust,
-                       "peak_burst": tc_burst, "frac_burst": tflops / tc_burst,
-                       "peak_nominal": TC_NOMINAL_TFLOPS,
-                       "frac_nominal": tflops / TC_NOMINAL_TFLOPS}}
+            "tensor": tensor}
     entry = {
         "metric": f"MoE-layer tokens/s ({cfg.name}, T={cfg.T})",
         "value": world * cfg.T / (ms_per_step * 1e-3),
@@ -527,7 +580,8 @@ def run_workload(name, args, world, local_rank, cache):
         "regions": len(region_ms),
         "region_ms": {"median": ms_region, "min": float(np.min(region_ms)),
                       "max": float(np.max(region_ms))},
-        "dtype": f"{cfg.fmt} weights, bf16 activations, fp32 accumulate",
+        "dtype": (f"{cfg.fmt} weights, bf16 activations, fp32 accumulate" if not nv else
+                  "nvfp4 weights and activations (routed), bf16 shared expert, fp32 accumulate"),
         "config": workload_config(cfg, world, args.replicas),
         "roofline": roof,
         "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s",

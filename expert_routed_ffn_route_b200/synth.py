@@ -46,7 +46,7 @@ __all__ = [
     "quantize_groups", "derive_seed", "FMT_BITS", "plant_ties",
 ]
 
-FMT_BITS = {"bf16": 16, "int8": 8, "int4": 4}
+FMT_BITS = {"bf16": 16, "int8": 8, "int4": 4, "nvfp4": 4}
 
 
 @dataclass(frozen=True)
@@ -76,6 +76,11 @@ CONFIGS = {
     "prefill": LayerConfig("prefill", T=512, d=2560, E=512, k=10, f=1024, fmt="int4"),
     "long": LayerConfig("long", T=4096, d=2560, E=512, k=10, f=1024, fmt="int8",
                         zipf_s=1.1),
+    # the W4A4 variant (NVFP4 routed experts, BF16 shared expert) on the prefill shapes
+    "prefill_nvfp4": LayerConfig("prefill_nvfp4", T=512, d=2560, E=512, k=10, f=1024,
+                                 fmt="nvfp4", shared_fmt="bf16"),
+    "long_nvfp4": LayerConfig("long_nvfp4", T=4096, d=2560, E=512, k=10, f=1024, fmt="nvfp4",
+                              shared_fmt="bf16", zipf_s=1.1),
 }
 
 
