@@ -536,6 +536,7 @@ def run_workload(name, args, world, local_rank, cache):
     e2e_ms = e0.elapsed_time(e1) / e_steps
     (e2e_ms,) = max_over_ranks([e2e_ms], device=dev)
     status = B.device_status(descs[0], ws)
+    site = B.device_wait_site(descs[0], ws) if status else 0
 
     hbm, tc_burst, tc_sust, peak_kind = measured_peaks()
     lb = float(np.mean(layer_bytes))
@@ -590,6 +591,8 @@ def run_workload(name, args, world, local_rank, cache):
         "clocks": clk.summary(),
         "device_status": status,
     }
+    if status:
+        entry["device_wait_site"] = site
     if cfg.T >= 512:  # the tensor-core workloads: the contraction's share of the roofline
         roof["tc_frac"] = roof["tensor"]["frac"]
     del layers, base, descs, ws, x_dev

@@ -48,7 +48,7 @@ EXPORTS = ["moe_abi_version", "moe_status_str", "moe_validate", "moe_workspace_s
            "moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
            "moe_layer_forward_marked", "moe_device_status", "moe_launches_per_call",
            "moe_layer_forward_static", "moe_static_device_status", "moe_test_inject_hold",
-           "moe_nvfp4_pack_scales", "moe_nvfp4_quantize_rows"]
+           "moe_nvfp4_pack_scales", "moe_nvfp4_quantize_rows", "moe_device_wait_site"]
 
 
 def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
@@ -78,6 +78,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "moe_layer_forward_marked": (I32, [LP, P, P, P, P, P, P, P, SZ, P,
                                            ctypes.POINTER(P), I32]),
         "moe_device_status": (I32, [LP, P, SZ, ctypes.POINTER(I32), P]),
+        "moe_device_wait_site": (I32, [LP, P, SZ, ctypes.POINTER(I32), P]),
         "moe_launches_per_call": (I32, [LP]),
         "moe_layer_forward_static": (I32, [LP, P, P, P]),
         "moe_static_device_status": (I32, [ctypes.POINTER(I32), P]),
@@ -288,6 +289,15 @@ def device_status(L: MoeLayer, ws, stream=None) -> int:
                                             ctypes.byref(code), _stream(stream)),
            "moe_device_status")
     return code.value
+
+
+def device_wait_site(L: MoeLayer, ws, stream=None) -> int:
+    """Site of the first device-side wait that gave up since the last read (0: none)."""
+    site = ctypes.c_int32(0)
+    _check(load_library().moe_device_wait_site(ctypes.byref(L), ws.data_ptr(), ws.numel(),
+                                               ctypes.byref(site), _stream(stream)),
+           "moe_device_wait_site")
+    return site.value
 
 
 def layer_forward_static(L: MoeLayer, x, out=None, stream=None):

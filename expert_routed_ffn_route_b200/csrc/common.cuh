@@ -44,6 +44,18 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, DEV_OK, code);
 }
 
+// Word 2 of the status block (byte 8 of the synchronisation block) keeps the site of the
+// first bounded wait that gave up (kernel and wait, numbered in include/moe_b200.h).
+constexpr int kSiteWord = 2;
+
+// A bounded wait at `site` gave up: DEV_TIMEOUT in the status word, the site beside it (the
+// first failure of a call wins both words).
+__device__ __forceinline__ void set_timeout(int32_t* status, int32_t site) {
+  if (!status) return;
+  atomicCAS(status, DEV_OK, DEV_TIMEOUT);
+  atomicCAS(status + kSiteWord, 0, site);
+}
+
 // ------------------------------------------------------------------ stable top-k
 
 // Order-preserving map of a finite float to uint32 (larger float -> larger key); -0 and
@@ -188,8 +200,8 @@ struct TcSched {
   int32_t* expert_mt;    // [E + 2]
 };
 
-// The synchronisation block at the start of the workspace: status word (offset 0), routing
-// tickets (16, 20), the single-kernel layer's grid-barrier word (32), the failure-injection
+// The synchronisation block at the start of the workspace: status word (offset 0), the site
+// of the first expired wait (8), routing tickets (16, 20), the single-kernel layer's grid-barrier word (32), the failure-injection
 // words (64: hold, 68: wait budget; zero in normal use), then one arrival counter per 16-row
 // output tile (256).
 constexpr size_t kSyncStatus = 0, kSyncTicket = 16, kSyncGbar = 32, kSyncTest = 64,

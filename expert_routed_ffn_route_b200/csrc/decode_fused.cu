@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       if (lane == 0) s_xsum[g] = s;
     }
     if (!mbar_wait(bar_router, 0)) {
-      set_status(p.status, DEV_TIMEOUT);
+      set_timeout(p.status, 20);
       mi->ok = 0;
     }
     for (int g = warp; g < G; g += kDfWarps) {
@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     for (int b = b_begin; b < b_end; ++b) {
       if (warp >= 2 * G) break;
       if (!warp_wait(&bar_tile[b])) {
-        if (lane == 0) set_status(p.status, DEV_TIMEOUT);
+        if (lane == 0) set_timeout(p.status, 21);
         return;
       }
       const uint8_t* tile = smem + (size_t)b * L.tile_bytes;
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     if (lane == 0) {
       s_arrived = gbar_arrive(gbar);
       if (mi->ok && (!gbar_wait(gbar, s_arrived) || !test_hold_wait(p.test_ctl))) {
-        set_status(p.status, DEV_TIMEOUT);
+        set_timeout(p.status, 22);
         mi->ok = 0;
       }
     }
@@ -632,7 +632,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     if (lane == 0) {
       s_arrived = gbar_arrive(gbar);
       if (ok1 && !gbar_wait(gbar, s_arrived)) {
-        set_status(p.status, DEV_TIMEOUT);
+        set_timeout(p.status, 23);
         mi->ok = 0;
       }
       if (mi->ok) {  // every h row of the call, into shared memory in one request
@@ -668,7 +668,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       const int first = ((warp - (u - u_begin) * Gf) % kDfWarps + kDfWarps) % kDfWarps;
       if (first >= Gf) continue;
       if (!warp_wait(&bar_unit[u])) {
-        if (lane == 0) set_status(p.status, DEV_TIMEOUT);
+        if (lane == 0) set_timeout(p.status, 24);
         return;
       }
       for (int g = first; g < Gf; g += kDfWarps) {
@@ -740,7 +740,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     bool ready = false;
     if (ok2) {
       ready = warp_wait(bar_h);
-      if (!ready && lane == 0) set_status(p.status, DEV_TIMEOUT);
+      if (!ready && lane == 0) set_timeout(p.status, 25);
       // h rows -> fragment order in place, and their per-group sums (a half-warp a group:
       // each lane one 8-value chunk, then a fixed tree over the 16 chunks)
       const int n_groups = S * Gf;

@@ -11,7 +11,10 @@
 //
 // Work: tiles (active expert, ROWS rows) in a flat list; CTA c (one per SM, persistent)
 // takes a contiguous range, so consecutive tiles mostly share an expert and its staged
-// activation rows. Each weight byte is read from HBM once per call; tokens beyond 8 for one
+// activation rows. Ranges are balanced by cost, a shared-expert tile (T rows) weighing its
+// token chunks: with equal tile counts, the CTAs holding the shared expert's tiles took
+// T / 8 times longer than the rest (measured on B200: 16 and 32 rows ran 2x and 4x slower
+// than 8 rows per expert tile predicted). Each weight byte is read from HBM once per call; tokens beyond 8 for one
 // expert re-use the staged tile from shared memory.
 //
 // What is computed is the same as gemv_ffn.cu: h = silu(Wg x) * (Wu x) per grouped row
@@ -148,9 +151,19 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
 
   const int n_active = p.active[0];
   const int n_rowtiles = N / Sh::ROWS;
-  const int n_tiles = (n_active + (p.has_shared ? 1 : 0)) * n_rowtiles;
-  const int t_begin = (int)((long long)n_tiles * blockIdx.x / gridDim.x);
-  const int t_end = (int)((long long)n_tiles * (blockIdx.x + 1) / gridDim.x);
+  // Contiguous tile ranges balanced by cost: a routed tile (a few rows) costs 1, a shared-
+  // expert tile (all T rows) costs its kTok-row chunks. A CTA takes the tiles whose cost
+  // interval starts inside its share [c0, c1) of the total (the partition moves no
+  // arithmetic: every tile is computed the same way whichever CTA takes it).
+  const int n_rt = n_active * n_rowtiles;
+  const int n_st = p.has_shared ? n_rowtiles : 0;
+  const int s_cost = (p.T + kTok - 1) / kTok;
+  const long long total_cost = (long long)n_rt + (long long)n_st * s_cost;
+  auto first_tile = [&](long long c) -> int {
+    return c <= n_rt ? (int)c : n_rt + (int)((c - n_rt + s_cost - 1) / s_cost);
+  };
+  const int t_begin = first_tile(total_cost * blockIdx.x / gridDim.x);
+  const int t_end = first_tile(total_cost * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == kCons) {
     // ------------------------------------------------------------ producer
@@ -159,7 +172,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
       for (int ti = t_begin; ti < t_end; ++ti, ++i) {
         const int s = i % Sh::NS, u = i / Sh::NS;
         if (u > 0 && !mbar_wait(&empty[s], (u - 1) & 1)) {
-          set_status(p.status, DEV_TIMEOUT);
+          set_timeout(p.status, 30);
           break;
         }
         const TileInfo t = tile_info(p, ti, n_rowtiles, n_active);
@@ -200,7 +213,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
     if (ctid == 0) flag[1] = mbar_wait(&full[s], u & 1) ? 1 : 0;
     named_bar_sync(1, 32 * kCons);
     if (!flag[1]) {
-      if (ctid == 0) set_status(p.status, DEV_TIMEOUT);
+      if (ctid == 0) set_timeout(p.status, 31);
       break;
     }
     if (pre) {

@@ -489,6 +489,22 @@ moe_status moe_nvfp4_quantize_rows(const float* v, int32_t rows, int32_t K, void
   return MOE_OK;
 }
 
+moe_status moe_device_wait_site(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* site,
+                                moe_stream_t stream) {
+  moe_status s = validate(L);
+  if (s != MOE_OK) return s;
+  if (!site) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(L, ws, ws_bytes)) != MOE_OK) return s;
+  int32_t* dev = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + layout(L).status) + kSiteWord;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  MOE_TRY(cudaMemcpyAsync(&h, dev, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  MOE_TRY(cudaStreamSynchronize(st));
+  MOE_TRY(cudaMemsetAsync(dev, 0, sizeof(int32_t), st));
+  *site = h;
+  return MOE_OK;
+}
+
 moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,
                              moe_stream_t stream) {
   moe_status s = validate(L);

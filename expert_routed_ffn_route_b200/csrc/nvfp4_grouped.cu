@@ -385,8 +385,8 @@ __global__ void __launch_bounds__(kNvThreads, 1)
   }
   __syncthreads();
   const int total = Ss.mt_prefix[n_active] * n_tiles;  // routed units only
-  auto fail = [&]() {
-    set_status(p.status, DEV_TIMEOUT);
+  auto fail = [&](int site) {
+    set_timeout(p.status, site);
     *abort_flag = 1;
   };
 
@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
                    C::SF_BYTES, &full[s]);
         }
       }
-      if (!ok) fail();
+      if (!ok) fail(40);
       // every issued stage lands before the CTA may exit
       for (int j = (it > C::NS ? it - C::NS : 0); j < it; ++j)
         mbar_wait(&full[j % C::NS], (j / C::NS) & 1);
@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       if (aborted) break;
       umma_commit_warp(&acc_full[b]);
     }
-    if (aborted) fail();
+    if (aborted) fail(41);
     // all issued MMAs and copies complete before TMEM and shared memory are released
     umma_commit_warp(drain);
     mbar_wait(drain, 0);
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(kNvThreads, 1)
       const TcUnit t = tc_unit(Ss, n_active, n_tiles, u);
       const int b = tile & 1;
       if (!mbar_wait(&acc_full[b], (tile >> 1) & 1)) {
-        fail();
+        fail(42);
         break;
       }
       tc_fence_after();

@@ -111,9 +111,9 @@ __global__ void __launch_bounds__(kRFThreads) route_fused_kernel(Plan p, int32_t
   }
   if (threadIdx.x == 0) {
     if (!gbar_wait(reinterpret_cast<const uint32_t*>(&ticket[0]), s_arrived))
-      set_status(p.status, DEV_TIMEOUT);
+      set_timeout(p.status, 1);
     else if (!test_hold_wait(p.test_ctl))
-      set_status(p.status, DEV_TIMEOUT);
+      set_timeout(p.status, 2);
   }
   __syncthreads();
   __threadfence();

@@ -400,8 +400,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int u_begin = (part == 2) ? Ss.mt_prefix[n_active] * n_tiles : 0;
   const int total = (part == 1) ? Ss.mt_prefix[n_active] * n_tiles : Ss.mt_prefix[n_slots] * n_tiles;
 
-  auto fail = [&]() {
-    set_status(p.status, DEV_TIMEOUT);
+  auto fail = [&](int site) {
+    set_timeout(p.status, site);
     *abort_flag = 1;
   };
 
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // the unit's group scales: kTcM consecutive rows, one contiguous block per matrix
           const int sbuf = ui & 1;
           if (ui >= 2 && !mbar_wait(&scale_empty[sbuf], ((ui >> 1) - 1) & 1)) {
-            fail();
+            fail(10);
             break;
           }
           mbar_arrive_expect_tx(&scale_full[sbuf], (uint32_t)(NM * SL.sb));
@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         cw * C::RAW_ROW, wrow, &full_w[sw]);
         }
         if (!ok) {
-          fail();
+          fail(11);
           break;
         }
       }
@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int b = tile % C::ACC_BUFS, buse = tile / C::ACC_BUFS;
       aborted = aborted || *abort_flag;
       if (!aborted && buse > 0 && !mbar_wait(&acc_empty[b], (buse - 1) & 1)) {
-        fail();
+        fail(12);
         aborted = true;
       }
       aborted = __any_sync(0xffffffffu, aborted);
@@ -532,7 +532,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       aborted = aborted || *abort_flag;
       if constexpr (FMT != 16) {
         if (!aborted && !mbar_wait(&scale_full[sbuf], (ui >> 1) & 1)) {
-          fail();
+          fail(13);
           aborted = true;
         }
       }
@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // every warp waits for every stage before releasing it (keeps the release phases
         // of the stage in order, also for a group with no chunk in it)
         if (!aborted && !mbar_wait(&full_w[sw], (it / C::NW) & 1)) {
-          fail();
+          fail(14);
           aborted = true;
         }
         aborted = __any_sync(0xffffffffu, aborted);
@@ -556,11 +556,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // the stage's previous chunk is consumed (waited for also after a failure; the
             // issuers never stop, so this wait ends)
             if (ia + j >= C::NA && !mbar_wait(&empty_x[a], (((ia + j) / C::NA) - 1) & 1)) {
-              fail();
+              fail(15);
               aborted = true;
             }
             if (!aborted && !mbar_wait(&full_x[a], ((ia + j) / C::NX) & 1)) {
-              fail();
+              fail(16);
               aborted = true;
             }
           }
@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       &full_x[sx]);
         }
         if (!ok) {
-          fail();
+          fail(17);
           break;
         }
       }
@@ -635,7 +635,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const TcUnit t = tc_unit(Ss, n_slots, n_tiles, u);
       const int b = tile % C::ACC_BUFS;
       if (!mbar_wait(&acc_full[b], (tile / C::ACC_BUFS) & 1)) {
-        fail();
+        fail(18);
         break;
       }
       tc_fence_after();

@@ -197,6 +197,19 @@ MOE_API int32_t moe_launches_per_call(const moe_layer* L);
 MOE_API moe_status moe_device_status(const moe_layer* L, void* ws, size_t ws_bytes, int32_t* code,
                              moe_stream_t stream);
 
+/* Where a MOE_ERR_TIMEOUT came from: the site of the first bounded device-side wait that gave
+ * up since the last read (0: none), read from the workspace and cleared (synchronises
+ * `stream`). Sites: 1 fused routing grid barrier, 2 fused routing test hold; 10..18 integer/
+ * bf16 tensor-core GEMMs (10 scale buffer free, 11 weight stage free, 12 accumulator free,
+ * 13 scales landed, 14 weight stage landed, 15 operand stage free, 16 activation stage landed,
+ * 17 activation stage free (producer), 18 accumulator full); 20..25 single-kernel 1-token
+ * layer (20 router rows landed, 21 gate/up tile landed, 22 first grid barrier, 23 second grid
+ * barrier, 24 down unit landed, 25 h rows landed); 30 TMA GEMV stage free, 31 TMA GEMV stage
+ * landed; 40..42 NVFP4 GEMMs (40 stage free, 41 accumulator free or stage landed, 42
+ * accumulator full). */
+MOE_API moe_status moe_device_wait_site(const moe_layer* L, void* ws, size_t ws_bytes,
+                                        int32_t* site, moe_stream_t stream);
+
 /* Failure injection, for tests of the error path: sets (hold != 0) or clears (hold == 0)
  * the hold word in the workspace's synchronisation block, with a wait budget in SM clock
  * cycles (0 = the library's normal bound of about two seconds). While the word is set, the

@@ -33,8 +33,10 @@ def B():
     return binding
 
 
-@pytest.mark.parametrize("T,path,launches", [(1, "fused", 1), (5, "gemv", None)])
-def test_bounded_wait_runs_out_and_is_reported(B, T, path, launches):
+# the wait sites the hold reaches (moe_device_wait_site): the single-kernel layer's first
+# grid barrier, the fused routing kernel's test hold
+@pytest.mark.parametrize("T,path,launches,site", [(1, "fused", 1, 22), (5, "gemv", None, 2)])
+def test_bounded_wait_runs_out_and_is_reported(B, T, path, launches, site):
     cfg = synth.LayerConfig("hold", T=T, d=2048, E=64, k=8, f=1024, fmt="int4", seed=43)
     L = synth.make_layer(cfg)
     dl = B.DeviceLayer(L)
@@ -54,6 +56,8 @@ def test_bounded_wait_runs_out_and_is_reported(B, T, path, launches):
     torch.cuda.synchronize()
     assert B.device_status(desc, ws) == MOE_ERR_TIMEOUT
     assert B.device_status(desc, ws) == 0  # read and cleared
+    assert B.device_wait_site(desc, ws) == site
+    assert B.device_wait_site(desc, ws) == 0
 
     # the same workspace, hold cleared: its barrier words and counters are consistent
     B.test_inject_hold(desc, ws, False)
@@ -61,6 +65,7 @@ def test_bounded_wait_runs_out_and_is_reported(B, T, path, launches):
         out = B.layer_forward(desc, x, ws)
         torch.cuda.synchronize()
         assert B.device_status(desc, ws) == 0
+        assert B.device_wait_site(desc, ws) == 0
         assert matches_oracle(out)
 
     # a fresh workspace
