@@ -171,6 +171,8 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
   pdl_wait();
   if (blockIdx.x == 0) {
     __shared__ int s_units[kMaxE + 1];
+    __shared__ int s_exp[kMaxE + 1];
+    __shared__ int s_warp[8];
     const int n_active = p.active[0];
     const int n_slots = n_active + (p.has_shared ? 1 : 0);
     for (int s = threadIdx.x; s < n_slots; s += blockDim.x) {
@@ -188,17 +190,34 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Plan p, TcSched S, uint16_
       S.slot_row0[s] = row0;
       S.slot_expert[s] = e;
       s_units[s] = (rows + kTcNMax - 1) / kTcNMax;  // m-tiles of the slot
+      s_exp[s] = e;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {  // serial prefix over at most E + 1 slots
-      int run = 0;
-      for (int s = 0; s < n_slots; ++s) {
-        S.mt_prefix[s] = run;
-        if (s < n_active) S.expert_mt[S.slot_expert[s]] = run;
-        run += s_units[s];
-      }
-      S.mt_prefix[n_slots] = run;
+    // exclusive prefix of the m-tiles over the slots: thread i sums a run of `per` slots,
+    // the runs are scanned across the block, then each thread writes its run's prefixes
+    const int per = (n_slots + blockDim.x - 1) / blockDim.x;
+    const int s0 = min(n_slots, (int)threadIdx.x * per), s1 = min(n_slots, s0 + per);
+    int local = 0;
+    for (int s = s0; s < s1; ++s) local += s_units[s];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
+    if (lane == 31) s_warp[wid] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < wid; ++w) base += s_warp[w];
+    int run = base + incl - local;
+    for (int s = s0; s < s1; ++s) {
+      S.mt_prefix[s] = run;
+      if (s < n_active) S.expert_mt[s_exp[s]] = run;
+      run += s_units[s];
+    }
+    if (s1 == n_slots && s0 < s1) S.mt_prefix[n_slots] = run;
+    if (n_slots == 0 && threadIdx.x == 0) S.mt_prefix[0] = 0;
   }
   {
     // one row per warp, lanes over the row's 16-byte pieces: the source token and the K order
