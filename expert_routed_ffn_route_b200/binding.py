@@ -184,9 +184,13 @@ def workspace_size(L: MoeLayer) -> int:
 
 
 def alloc_workspace(L: MoeLayer, device="cuda"):
-    """A zeroed workspace (the status word at its start must begin at zero)."""
+    """A zeroed workspace (the status word at its start must begin at zero). The fill is
+    waited for here, so the workspace may be used on any stream: a fill still queued behind
+    other work while a call runs on another stream would reset the call's barrier words."""
     import torch
-    return torch.zeros(workspace_size(L), dtype=torch.uint8, device=device)
+    ws = torch.zeros(workspace_size(L), dtype=torch.uint8, device=device)
+    torch.cuda.current_stream(ws.device).synchronize()
+    return ws
 
 
 def route(L: MoeLayer, x, ws, stream=None):

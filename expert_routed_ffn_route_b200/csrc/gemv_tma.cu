@@ -28,7 +28,6 @@
 
 namespace moe {
 
-#define TRACE(slot) do {} while (0)
 
 constexpr int kCons = 16;                    // consumer warps
 constexpr int kTmaThreads = 32 * (kCons + 1);  // + one producer warp
@@ -257,9 +256,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
       for (int mi = 0; mi < NM; ++mi)
 #pragma unroll
         for (int q = 0; q < 4; ++q) myred[mi * 4 + q] = acc[mi][q];
-      TRACE(tr++);
       named_bar_sync(1, 32 * kCons);
-      TRACE(tr++);
       // fixed-order sum over the K split, then the epilogue
       for (int o = ctid; o < Sh::ROWS * kTok; o += 32 * kCons) {
         const int row = o / kTok, tok = o % kTok;
@@ -287,7 +284,6 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
         }
       }
       named_bar_sync(1, 32 * kCons);
-      TRACE(tr++);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
