@@ -125,11 +125,11 @@ __host__ __device__ inline DfLayout df_layout(int grid, int d, int f, int E, int
     L.off_ybuf = o;
     o += ybuf_bytes;
   }
+  // K-split partials: [tile][matrix][split part][16 rows], then [unit][split part][16 rows]
   L.off_red = o;
-  uint32_t red_gu = (uint32_t)L.tiles_max * 2 * L.G * kDfRows * 4;
-  uint32_t red_dn = (uint32_t)L.units_max * L.Gf * kDfRows * 4;
-  uint32_t red_rt = (uint32_t)kDfMaxRouter * L.G * 4;
-  o += max(red_gu, max(red_dn, red_rt));
+  uint32_t red_gu = (uint32_t)L.tiles_max * 2 * kKsGateUp * kDfRows * 4;
+  uint32_t red_dn = (uint32_t)L.units_max * kKsDown * kDfRows * 4;
+  o += max(red_gu, red_dn);
   o = (o + 15) & ~15u;
   L.off_bar = o;
   o += 8u * (2 + kDfMaxTiles + kDfMaxUnits);
@@ -154,7 +154,9 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 // One 128-wide K group of a 16-row int4 tile against one activation row held as the
 // B operand's column 0 (xb: the lane's 32 activation values of the group, permuted into
 // fragment order; zero on lanes that do not carry column 0). Returns, on lanes with q == 0,
-// the biased dot products of rows grp and grp + 8 (codes enter as q + 136).
+// the biased dot products of rows grp and grp + 8 (codes enter as q + 136). The 8 MMAs of
+// the group accumulate in one chain, in the order the GEMV kernels use (gemv_frag.cuh), so
+// the group product is the same bits as theirs.
 __device__ __forceinline__ void t1_group(const uint8_t* tile, uint32_t row_bytes, int g, int grp,
                                          int q, const uint32_t (&xb)[16], float& ra,
                                          float& rb) {
@@ -164,15 +166,12 @@ __device__ __forceinline__ void t1_group(const uint8_t* tile, uint32_t row_bytes
   uint32_t fa[8][2], fb[8][2];
   to_frags<4>(wa, fa);
   to_frags<4>(wb, fb);
-  float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int m = 0; m < 8; m += 2) {
-    mma_bf16_16x8x16(c0, fa[m][0], fb[m][0], fa[m][1], fb[m][1], xb[2 * m], xb[2 * m + 1]);
-    mma_bf16_16x8x16(c1, fa[m + 1][0], fb[m + 1][0], fa[m + 1][1], fb[m + 1][1],
-                     xb[2 * m + 2], xb[2 * m + 3]);
-  }
-  ra = c0[0] + c1[0];
-  rb = c0[2] + c1[2];
+  for (int m = 0; m < 8; ++m)
+    mma_bf16_16x8x16(c, fa[m][0], fb[m][0], fa[m][1], fb[m][1], xb[2 * m], xb[2 * m + 1]);
+  ra = c[0];
+  rb = c[2];
 }
 
 // The lane's 32 activation values [32 q, 32 q + 32) of group g of a bf16 row, in fragment
@@ -319,87 +318,97 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
 
   // ---------------------------------------------------------------- router logits
   if (!producer) {
-    for (int g = warp; g < G; g += kDfWarps) {  // per-group sums of x
-      const uint2 v = *reinterpret_cast<const uint2*>(s_x + g * kGroup + 4 * lane);
-      float s = __uint_as_float(v.x << 16);
-      s += __uint_as_float(v.x & 0xffff0000u);
-      s += __uint_as_float(v.y << 16);
-      s += __uint_as_float(v.y & 0xffff0000u);
+    // per-group sums of x as the GEMV kernels stage them: a half-warp a group, lane l the 8
+    // values of 16-byte chunk l in order, then a fixed tree over the 16 chunks (the value of
+    // chunk 0's lane); both half-warps run every pass, so the shuffles stay warp-uniform
+    for (int pi = warp; pi < (G + 1) / 2; pi += kDfWarps) {
+      const int gi = 2 * pi + (lane >> 4);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (gi < G) v = reinterpret_cast<const uint4*>(s_x + gi * kGroup)[lane & 15];
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+      float sm = 0.f;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) s_xsum[g] = s;
+      for (int j = 0; j < 4; ++j) {
+        sm += __uint_as_float(vv[j] << 16);
+        sm += __uint_as_float(vv[j] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+      if (gi < G && (lane & 15) == 0) s_xsum[gi] = sm;
     }
     if (!mbar_wait(bar_router, 0)) {
       set_timeout(p.status, 20);
       mi->ok = 0;
     }
-    for (int g = warp; g < G; g += kDfWarps) {
-      const uint2 xv = *reinterpret_cast<const uint2*>(s_x + g * kGroup + 4 * lane);
-      const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
-      const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
-      float s[kDfMaxRouter];
+    // logits in the order of the fused routing kernel (route_fused.cu), so a token's logits
+    // and gates are the same bits whichever of the two kernels routes it: lane l takes the
+    // 16-byte pieces l, l + 32, ... of the row in batches of 8 (pieces past the row are
+    // zeros), one fused multiply-add chain over each piece's 8 values in order, then a fixed
+    // tree over the lanes, then the bias
+    const int n16 = d / 8;
+    const uint4* xrow = reinterpret_cast<const uint4*>(s_x);
+    for (int r = warp; r < nr; r += kDfWarps) {
+      const uint4* wrow = reinterpret_cast<const uint4*>(s_router + (size_t)r * d);
+      float acc = 0.f;
+      for (int c0 = 0; c0 < n16; c0 += 8 * 32) {
 #pragma unroll
-      for (int r = 0; r < kDfMaxRouter; ++r) {
-        s[r] = 0.f;
-        if (r < nr) {
-          const uint2 wv = *reinterpret_cast<const uint2*>(s_router + (size_t)r * d + g * kGroup + 4 * lane);
-          s[r] = x0 * __uint_as_float(wv.x << 16);
-          s[r] = fmaf(x1, __uint_as_float(wv.x & 0xffff0000u), s[r]);
-          s[r] = fmaf(x2, __uint_as_float(wv.y << 16), s[r]);
-          s[r] = fmaf(x3, __uint_as_float(wv.y & 0xffff0000u), s[r]);
+        for (int i = 0; i < 8; ++i) {
+          const int cc = c0 + lane + 32 * i;
+          const uint4 wv = (cc < n16) ? wrow[cc] : make_uint4(0, 0, 0, 0);
+          const uint4 xv = (cc < n16) ? xrow[cc] : make_uint4(0, 0, 0, 0);
+          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+          const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            acc = fmaf(__uint_as_float(xx[q4] << 16), __uint_as_float(ww[q4] << 16), acc);
+            acc = fmaf(__uint_as_float(xx[q4] & 0xffff0000u), __uint_as_float(ww[q4] & 0xffff0000u),
+                       acc);
+          }
         }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int r = 0; r < kDfMaxRouter; ++r) s[r] += __shfl_xor_sync(0xffffffffu, s[r], o);
-      if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < kDfMaxRouter; ++r)
-          if (r < nr) red[r * G + g] = s[r];
-      }
-    }
-    named_bar_sync(1, kDfCompute);
-    for (int r = warp; r < nr; r += kDfWarps) {  // a warp a row: fixed-order tree over groups
-      float s = 0.f;
-      for (int g = lane; g < G; g += 32) s += red[r * G + g];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       const int e = r0 + r;
-      if (lane == 0) p.logits[e] = s + (p.router_bias ? p.router_bias[e] : 0.f);
+      if (lane == 0) p.logits[e] = acc + (p.router_bias ? p.router_bias[e] : 0.f);
     }
   }
   __syncthreads();  // S2: this CTA's logits are written
 
-  // Items (tile position b, matrix m, group g), warp w takes every kDfWarps-th item of a
-  // tile range; partials land in red[b][m][g][16] (rows of the tile), scaled and corrected.
+  // Items (tile position b, K-split part ks) over the tile range, in tile-major order; warp w
+  // takes every kDfWarps-th. An item is part ks of both matrices of its tile: groups ks,
+  // ks + kKsGateUp, ..., each added to the part's partial as a fused multiply-add of the
+  // row's group scale and (group product - 136 x group sum of x), exactly as the GEMV kernels
+  // accumulate a row (gemv_frag.cuh). Partials land in red[b][m][ks][16 rows].
   auto gate_up_items = [&](int b_begin, int b_end) {
-    int cur_g = -1;
     uint32_t xb[16];
-    float corr = 0.f;
-    for (int b = b_begin; b < b_end; ++b) {
-      if (warp >= 2 * G) break;
+    const int n_items = (b_end - b_begin) * kKsGateUp;
+    for (int it = warp; it < n_items; it += kDfWarps) {
+      const int b = b_begin + it / kKsGateUp, ks = it % kKsGateUp;
       if (!warp_wait(&bar_tile[b])) {
         if (lane == 0) set_timeout(p.status, 21);
         return;
       }
       const uint8_t* tile = smem + (size_t)b * L.tile_bytes;
       const uint16_t* scales = reinterpret_cast<const uint16_t*>(tile + 2 * kDfRows * rowb_up);
-      float* red_b = red + (size_t)b * 2 * G * kDfRows;
-      for (int r = warp; r < 2 * G; r += kDfWarps) {
-        const int m = (r >= G) ? 1 : 0, g = r - m * G;
-        if (g != cur_g) {
-          t1_load_act<false>(s_x, g, q, grp == 0, xb);
-          corr = 136.f * s_xsum[g];
-          cur_g = g;
-        }
-        float ra, rb;
-        t1_group(tile + m * kDfRows * rowb_up, rowb_up, g, grp, q, xb, ra, rb);
-        if (q == 0) {
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // [matrix][row grp, row grp + 8]
+      for (int g = ks; g < G; g += kKsGateUp) {
+        t1_load_act<false>(s_x, g, q, grp == 0, xb);
+        const float corr = 136.f * s_xsum[g];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          float ra, rb;
+          t1_group(tile + m * kDfRows * rowb_up, rowb_up, g, grp, q, xb, ra, rb);
           const uint16_t* sc = scales + m * kDfRows * G + g;
-          float* dst = red_b + (size_t)r * kDfRows;
-          dst[grp] = bf16_to_f32(sc[grp * G]) * (ra - corr);
-          dst[grp + 8] = bf16_to_f32(sc[(grp + 8) * G]) * (rb - corr);
+          acc[m][0] = fmaf(bf16_to_f32(sc[grp * G]), ra - corr, acc[m][0]);
+          acc[m][1] = fmaf(bf16_to_f32(sc[(grp + 8) * G]), rb - corr, acc[m][1]);
+        }
+      }
+      if (q == 0) {
+        float* red_b = red + (size_t)b * 2 * kKsGateUp * kDfRows;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          red_b[(m * kKsGateUp + ks) * kDfRows + grp] = acc[m][0];
+          red_b[(m * kKsGateUp + ks) * kDfRows + grp + 8] = acc[m][1];
         }
       }
     }
@@ -517,15 +526,12 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       }
     }
     named_bar_sync(1, kDfCompute);
-    if (warp == 0) {
+    if (warp == 0) {  // the gates as the routing kernels form them (warp_topk_gate)
       const uint32_t my_key = (lane < k) ? reinterpret_cast<const uint32_t*>(mi->gate)[lane] : 0u;
       const uint32_t top = __shfl_sync(0xffffffffu, my_key, 0);
-      const float z = (lane < k) ? expf(key_value(my_key) - key_value(top)) : 0.f;
-      float tot = z;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      const float gate = warp_topk_gate(my_key, top, k, lane);
       __syncwarp();
-      if (lane < k) mi->gate[lane] = z / tot;
+      if (lane < k) mi->gate[lane] = gate;
     }
   }
   __syncthreads();  // S4: the routing decision
@@ -610,15 +616,16 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
     }
     __syncwarp();
   } else if (ok1) {
-    // h rows of this CTA's tiles: fixed-order sums over the K groups, SwiGLU, one rounding
+    // h rows of this CTA's tiles: the K-split partials added in part order (as the GEMV
+    // kernels add them), SwiGLU, one rounding
     for (int i = tid; i < mi->n_tiles * kDfRows; i += kDfCompute) {
       const int b = i / kDfRows, r = i % kDfRows;
-      const float* rg = red + (size_t)(b * 2) * G * kDfRows + r;
-      const float* ru = rg + (size_t)G * kDfRows;
+      const float* rg = red + (size_t)(b * 2) * kKsGateUp * kDfRows + r;
+      const float* ru = rg + (size_t)kKsGateUp * kDfRows;
       float gs = 0.f, us = 0.f;
-      for (int g = 0; g < G; ++g) {
-        gs += rg[g * kDfRows];
-        us += ru[g * kDfRows];
+      for (int ks = 0; ks < kKsGateUp; ++ks) {
+        gs += rg[ks * kDfRows];
+        us += ru[ks * kDfRows];
       }
       const float hv = gs / (1.f + expf(-gs)) * us;
       p.h[(size_t)mi->tile_slot[b] * f + (size_t)mi->tile_rt[b] * kDfRows + r] = f32_to_bf16_rn(hv);
@@ -658,20 +665,25 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
   // locally. Both combines sum the gates in rank order, then the shared term, in fp32.
   uint16_t* hw = reinterpret_cast<uint16_t*>(smem + L.off_h);
   float* s_hsum = reinterpret_cast<float*>(smem + L.off_hsum);
+  // Items (unit u, K-split part ks) in unit-major order from u_begin; warp w takes every
+  // kDfWarps-th (kDfWarps is a multiple of kKsDown, so at most one part of a unit each). Part
+  // ks sums groups ks, ks + kKsDown, ... as the GEMV kernels do; partials land in
+  // red[u][ks][16 rows].
+  static_assert(kDfWarps % kKsDown == 0, "one part of a unit per warp");
   auto down_items = [&](int u_begin, int u_end) {
     uint32_t xb[16];
     for (int u = u_begin; u < u_end; ++u) {
       const int slot = mi->unit_slot[u];
       const uint8_t* unit = smem + (size_t)u * L.unit_bytes;
       const uint16_t* scales = reinterpret_cast<const uint16_t*>(unit + kDfRows * rowb_dn);
-      // items (u, g) in u-major order from u_begin: warp w takes every kDfWarps-th
-      const int first = ((warp - (u - u_begin) * Gf) % kDfWarps + kDfWarps) % kDfWarps;
-      if (first >= Gf) continue;
+      const int ks = ((warp - (u - u_begin) * kKsDown) % kDfWarps + kDfWarps) % kDfWarps;
+      if (ks >= kKsDown) continue;
       if (!warp_wait(&bar_unit[u])) {
         if (lane == 0) set_timeout(p.status, 24);
         return;
       }
-      for (int g = first; g < Gf; g += kDfWarps) {
+      float acc0 = 0.f, acc1 = 0.f;
+      for (int g = ks; g < Gf; g += kKsDown) {
         const uint16_t* hrow = hw + (size_t)slot * f + g * kGroup + 32 * q;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -684,21 +696,22 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
         }
         float ra, rb;
         t1_group(unit, rowb_dn, g, grp, q, xb, ra, rb);
-        if (q == 0) {
-          const uint16_t* sc = scales + g;
-          const float corr = 136.f * s_hsum[slot * Gf + g];
-          float* dst = red + ((size_t)u * Gf + g) * kDfRows;
-          dst[grp] = bf16_to_f32(sc[grp * Gf]) * (ra - corr);
-          dst[grp + 8] = bf16_to_f32(sc[(grp + 8) * Gf]) * (rb - corr);
-        }
+        const float corr = 136.f * s_hsum[slot * Gf + g];
+        acc0 = fmaf(bf16_to_f32(scales[grp * Gf + g]), ra - corr, acc0);
+        acc1 = fmaf(bf16_to_f32(scales[(grp + 8) * Gf + g]), rb - corr, acc1);
+      }
+      if (q == 0) {
+        float* dst = red + ((size_t)u * kKsDown + ks) * kDfRows;
+        dst[grp] = acc0;
+        dst[grp + 8] = acc1;
       }
     }
   };
-  // y of unit u, row r: the fixed-order sum of its K-group partials
+  // y of unit u, row r: the K-split partials added in part order
   auto unit_y = [&](int u, int r) {
-    const float* src_r = red + (size_t)u * Gf * kDfRows + r;
+    const float* src_r = red + (size_t)u * kKsDown * kDfRows + r;
     float y = 0.f;
-    for (int g = 0; g < Gf; ++g) y += src_r[g * kDfRows];
+    for (int ks = 0; ks < kKsDown; ++ks) y += src_r[ks * kDfRows];
     return y;
   };
 
@@ -744,8 +757,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
       // h rows -> fragment order in place, and their per-group sums (a half-warp a group:
       // each lane one 8-value chunk, then a fixed tree over the 16 chunks)
       const int n_groups = S * Gf;
-      for (int gi = 2 * warp + (lane >> 4); gi < n_groups && ready; gi += 2 * kDfWarps) {
-        uint4* chunk = reinterpret_cast<uint4*>(hw + (size_t)gi * kGroup) + (lane & 15);
+      for (int pi = warp; pi < (n_groups + 1) / 2 && ready; pi += kDfWarps) {
+        const int gi = 2 * pi + (lane >> 4);  // both half-warps run every pass
+        uint4* chunk = reinterpret_cast<uint4*>(hw + (size_t)min(gi, n_groups - 1) * kGroup) +
+                       (lane & 15);
         uint4 v = *chunk;
         const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
         float s = 0.f;
@@ -755,10 +770,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) decode_fused_kernel(Plan p, uin
           s += __uint_as_float(vv[j] & 0xffff0000u);
         }
         permute_chunk<4>(v);
-        *chunk = v;
+        if (gi < n_groups) *chunk = v;
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if ((lane & 15) == 0) s_hsum[gi] = s;
+        if (gi < n_groups && (lane & 15) == 0) s_hsum[gi] = s;
       }
     }
     named_bar_sync(1, kDfCompute);

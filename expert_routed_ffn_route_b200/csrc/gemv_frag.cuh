@@ -16,6 +16,13 @@ namespace moe {
 
 constexpr int kTok = 8;       // tokens per MMA (N)
 
+// K split of one weight row's 128-wide groups: split part ks sums groups ks, ks + KS, ...
+// (a fused multiply-add chain of scale x (group product - offset correction)), and the
+// parts are added in ks order. The GEMV kernels and the single-kernel 1-token layer use the
+// same split, so a token's row comes out bit for bit the same whichever of them computes it.
+constexpr int kKsGateUp = 8;  // gate/up (K = d)
+constexpr int kKsDown = 4;    // down (K = f)
+
 template <int FMT> struct FmtInfo;
 template <> struct FmtInfo<4> { static constexpr int U = 1; static constexpr int bits = 4; };
 template <> struct FmtInfo<8> { static constexpr int U = 2; static constexpr int bits = 8; };

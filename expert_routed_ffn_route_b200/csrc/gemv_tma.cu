@@ -38,6 +38,7 @@ template <bool GATE_UP> struct TmaShape {
   static constexpr int RT = ROWS / 16;            // 16-row MMA tiles per tile
   static constexpr int KS = kCons / RT;           // consumer warps sharing one row tile (K split)
   static constexpr int NS = GATE_UP ? 2 : 5;      // pipeline stages
+  static_assert(KS == (GATE_UP ? kKsGateUp : kKsDown), "the shared K split (gemv_frag.cuh)");
 };
 
 struct TmaSmem {

@@ -10,7 +10,7 @@ using namespace moe;
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kTcMinTokens = 16;
+constexpr int kTcMinTokens = 33;
 inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -201,9 +201,14 @@ bool scales_aligned16(const Bank& b) {
 }
 
 // Grouped FFN kernels for the call: the tensor-core grouped GEMMs from kTcMinTokens tokens
-// up (measured on B200: 16- and 32-token verify calls run 1.5-1.9x faster there than on
-// the GEMV kernels), the TMA-pipelined GEMV for smaller int4 calls, the register-streaming
-// GEMV otherwise. Kernels after the first of a call use programmatic dependent launch.
+// up, the TMA-pipelined GEMV for smaller int4 calls, the register-streaming GEMV otherwise.
+// Up to 32 rows (decode and speculative-verify calls) the automatic choice keeps a token's
+// output bits independent of the call: the GEMV kernels and the single-kernel 1-token layer
+// share one arithmetic order (TandemLLM docs, "17 Qwen3.8-Flash-Next", §17.3: decode rows
+// must equal the rows of a verify chain bit for bit). The tensor cores would run 16- and
+// 32-row calls about 15% faster (measured on B200: 291 / 473 against 334 / 555 us) but sum
+// in another order; MOE_PATH_TC asks for them. Kernels after the first of a call use
+// programmatic dependent launch.
 bool use_tc(const Plan& p) {
   if (p.path == MOE_PATH_GEMV || p.path == MOE_PATH_FUSED) return false;
   if (p.path == MOE_PATH_TC) return true;
