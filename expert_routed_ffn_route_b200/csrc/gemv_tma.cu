@@ -32,25 +32,28 @@ namespace moe {
 constexpr int kCons = 16;                    // consumer warps
 constexpr int kTmaThreads = 32 * (kCons + 1);  // + one producer warp
 
-template <bool GATE_UP> struct TmaShape {
-  static constexpr int ROWS = GATE_UP ? 32 : 64;  // weight rows per tile
+// Tile shapes per weight format: int8 rows are twice as long, so its gate/up tiles have
+// half the rows (two stages still fit) and its down kernel two stages.
+template <int FMT, bool GATE_UP> struct TmaShape {
+  static constexpr int ROWS = GATE_UP ? (FMT == 4 ? 32 : 16) : 64;  // weight rows per tile
   static constexpr int NM = GATE_UP ? 2 : 1;      // matrices per tile
   static constexpr int RT = ROWS / 16;            // 16-row MMA tiles per tile
   static constexpr int KS = kCons / RT;           // consumer warps sharing one row tile (K split)
-  static constexpr int NS = GATE_UP ? 2 : 5;      // pipeline stages
-  static_assert(KS == (GATE_UP ? kKsGateUp : kKsDown), "the shared K split (gemv_frag.cuh)");
+  static constexpr int NS = GATE_UP ? 2 : (FMT == 4 ? 5 : 2);  // pipeline stages
+  // int4: the K split of the single-kernel 1-token layer, which computes the same rows
+  static_assert(FMT != 4 || KS == (GATE_UP ? kKsGateUp : kKsDown), "shared K split");
 };
 
 struct TmaSmem {
   size_t stage_bytes, w_bytes, s_bytes, xs_off, xsum_off, red_off, bar_off, flag_off, total;
 };
 
-template <bool GATE_UP>
+template <int FMT, bool GATE_UP>
 __host__ __device__ inline TmaSmem tma_smem_layout(int K) {
-  using Sh = TmaShape<GATE_UP>;
+  using Sh = TmaShape<FMT, GATE_UP>;
   TmaSmem m;
   const int G = K / kGroup;
-  m.w_bytes = (size_t)Sh::ROWS * K / 2;        // one matrix tile (int4)
+  m.w_bytes = (size_t)Sh::ROWS * K * FMT / 8;  // one matrix tile
   m.s_bytes = (size_t)Sh::ROWS * G * 2;        // its scales (bf16)
   m.stage_bytes = Sh::NM * (m.w_bytes + m.s_bytes);
   size_t o = Sh::NS * m.stage_bytes;
@@ -97,7 +100,7 @@ __device__ __forceinline__ TileInfo tile_info(const Plan& p, int ti, int n_rowti
 
 // Stage the activation rows of token chunk c0 of tile t (x gathered through perm for the
 // gate/up kernel, the h rows of the tile's expert for the down kernel).
-template <bool GATE_UP>
+template <int FMT, bool GATE_UP>
 __device__ __forceinline__ void stage_tile_rows(const Plan& p, const TileInfo& t, int c0, int K,
                                                 uint8_t* xs, int S, float* xsum, int ctid) {
   StageArgs sa;
@@ -115,19 +118,22 @@ __device__ __forceinline__ void stage_tile_rows(const Plan& p, const TileInfo& t
     sa.row0 = (t.shared ? p.T * p.k : 0) + t.row_begin + c0;
   }
   sa.nrows = min(kTok, t.nrows - c0);
-  stage_rows<4, 32 * kCons>(sa, K, xs, S, xsum, ctid);
+  stage_rows<FMT, 32 * kCons>(sa, K, xs, S, xsum, ctid);
 }
 
-template <bool GATE_UP>
-__global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
-  using Sh = TmaShape<GATE_UP>;
+// part: 0 every tile, 1 the routed experts' tiles, 2 the shared expert's (one launch per
+// bank when the banks' formats differ; FMT is the format of the tiles the launch takes).
+template <int FMT, bool GATE_UP>
+__global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p, int part) {
+  using Sh = TmaShape<FMT, GATE_UP>;
   constexpr int NM = Sh::NM;
+  constexpr int U = FmtInfo<FMT>::U;  // 16-byte pieces of a row's group a lane reads
   const int K = GATE_UP ? p.d : p.f;
   const int N = GATE_UP ? p.f : p.d;
   const int G = K / kGroup;
   const int S = 2 * K + 8;
-  const size_t row_bytes = (size_t)K / 2;
-  const TmaSmem L = tma_smem_layout<GATE_UP>(K);
+  const size_t row_bytes = (size_t)K * FMT / 8;
+  const TmaSmem L = tma_smem_layout<FMT, GATE_UP>(K);
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* xs = smem + L.xs_off;
@@ -155,15 +161,16 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
   // expert tile (all T rows) costs its kTok-row chunks. A CTA takes the tiles whose cost
   // interval starts inside its share [c0, c1) of the total (the partition moves no
   // arithmetic: every tile is computed the same way whichever CTA takes it).
-  const int n_rt = n_active * n_rowtiles;
-  const int n_st = p.has_shared ? n_rowtiles : 0;
+  const int n_rt = (part == 2) ? 0 : n_active * n_rowtiles;
+  const int n_st = (p.has_shared && part != 1) ? n_rowtiles : 0;
+  const int tile0 = (part == 2) ? n_active * n_rowtiles : 0;  // numbering of the full list
   const int s_cost = (p.T + kTok - 1) / kTok;
   const long long total_cost = (long long)n_rt + (long long)n_st * s_cost;
   auto first_tile = [&](long long c) -> int {
     return c <= n_rt ? (int)c : n_rt + (int)((c - n_rt + s_cost - 1) / s_cost);
   };
-  const int t_begin = first_tile(total_cost * blockIdx.x / gridDim.x);
-  const int t_end = first_tile(total_cost * (blockIdx.x + 1) / gridDim.x);
+  const int t_begin = tile0 + first_tile(total_cost * blockIdx.x / gridDim.x);
+  const int t_end = tile0 + first_tile(total_cost * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == kCons) {
     // ------------------------------------------------------------ producer
@@ -209,7 +216,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
     // The first token chunk of a new expert is staged before the wait for the tile's
     // weights, so the activation loads overlap the weight copies.
     const bool pre = (staged_slot != t.slot || staged_c0 != 0);
-    if (pre) stage_tile_rows<GATE_UP>(p, t, 0, K, xs, S, xsum, ctid);
+    if (pre) stage_tile_rows<FMT, GATE_UP>(p, t, 0, K, xs, S, xsum, ctid);
     if (ctid == 0) flag[1] = mbar_wait(&full[s], u & 1) ? 1 : 0;
     named_bar_sync(1, 32 * kCons);
     if (!flag[1]) {
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
       const int nr = min(kTok, t.nrows - c0);
       if (staged_slot != t.slot || staged_c0 != c0) {
         named_bar_sync(1, 32 * kCons);  // everyone is done with the previous rows
-        stage_tile_rows<GATE_UP>(p, t, c0, K, xs, S, xsum, ctid);
+        stage_tile_rows<FMT, GATE_UP>(p, t, c0, K, xs, S, xsum, ctid);
         named_bar_sync(1, 32 * kCons);
         staged_slot = t.slot;
         staged_c0 = c0;
@@ -239,18 +246,24 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p) {
         for (int q = 0; q < 4; ++q) acc[mi][q] = 0.f;
       const uint8_t* xrow = xs + (size_t)grp * S;
       for (int g = ks; g < G; g += Sh::KS) {
-        uint4 wa[NM][1], wb[NM][1];
+        uint4 wa[NM][U], wb[NM][U];
         float fsa[NM], fsb[NM];
 #pragma unroll
         for (int mi = 0; mi < NM; ++mi) {
           const uint8_t* wt = st + mi * L.w_bytes;
-          wa[mi][0] = *reinterpret_cast<const uint4*>(wt + la * row_bytes + g * 64 + q4 * 16);
-          wb[mi][0] = *reinterpret_cast<const uint4*>(wt + lb * row_bytes + g * 64 + q4 * 16);
+          // the lane's 32 K values of the group: 16 * U bytes of each of its two rows
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            wa[mi][u] = *reinterpret_cast<const uint4*>(wt + la * row_bytes + g * (16 * FMT) +
+                                                        q4 * (4 * FMT) + 16 * u);
+            wb[mi][u] = *reinterpret_cast<const uint4*>(wt + lb * row_bytes + g * (16 * FMT) +
+                                                        q4 * (4 * FMT) + 16 * u);
+          }
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(st + NM * L.w_bytes + mi * L.s_bytes);
           fsa[mi] = bf16_to_f32(sc[la * G + g]);
           fsb[mi] = bf16_to_f32(sc[lb * G + g]);
         }
-        group_mma<4, NM>(wa, wb, fsa, fsb, xrow, xsum, G, g, q4, acc);
+        group_mma<FMT, NM>(wa, wb, fsa, fsb, xrow, xsum, G, g, q4, acc);
       }
       float* myred = red + ((size_t)warp * 32 + lane) * (NM * 4);
 #pragma unroll
@@ -298,11 +311,11 @@ struct TmaLaunchCache {
   int sms = 0;
 };
 
-template <bool GATE_UP>
-static cudaError_t launch_tma(const Plan& p, cudaStream_t st, bool pdl) {
+template <int FMT, bool GATE_UP>
+static cudaError_t launch_tma_part(const Plan& p, int part, cudaStream_t st, bool pdl) {
   const int K = GATE_UP ? p.d : p.f;
-  const size_t smem = tma_smem_layout<GATE_UP>(K).total;
-  auto kern = gemv_tma_kernel<GATE_UP>;
+  const size_t smem = tma_smem_layout<FMT, GATE_UP>(K).total;
+  auto kern = gemv_tma_kernel<FMT, GATE_UP>;
   static TmaLaunchCache cache;
   int sms;
   {
@@ -330,14 +343,39 @@ static cudaError_t launch_tma(const Plan& p, cudaStream_t st, bool pdl) {
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, p, part);
+}
+
+template <bool GATE_UP>
+static cudaError_t launch_tma_fmt(const Plan& p, int fmt, int part, cudaStream_t st, bool pdl) {
+  return fmt == 8 ? launch_tma_part<8, GATE_UP>(p, part, st, pdl)
+                  : launch_tma_part<4, GATE_UP>(p, part, st, pdl);
+}
+
+// One launch when the banks share a format, else the routed experts and the shared expert
+// in two launches of their own formats (the second one after the first: same stream).
+template <bool GATE_UP>
+static cudaError_t launch_tma(const Plan& p, cudaStream_t st, bool pdl) {
+  if (!p.has_shared || p.shared.fmt == p.routed.fmt)
+    return launch_tma_fmt<GATE_UP>(p, p.routed.fmt, 0, st, pdl);
+  const cudaError_t err = launch_tma_fmt<GATE_UP>(p, p.routed.fmt, 1, st, pdl);
+  if (err != cudaSuccess) return err;
+  return launch_tma_fmt<GATE_UP>(p, p.shared.fmt, 2, st, true);
 }
 
 
+template <int FMT>
+static bool tma_fits(const Plan& p) {
+  return tma_smem_layout<FMT, true>(p.d).total <= 227 * 1024 &&
+         tma_smem_layout<FMT, false>(p.f).total <= 227 * 1024;
+}
+
+// int4 and int8 banks (in any pairing); bf16 banks take the register-streaming GEMV.
 bool tma_gemv_supported(const Plan& p) {
-  if (p.routed.fmt != 4 || (p.has_shared && p.shared.fmt != 4)) return false;
-  return tma_smem_layout<true>(p.d).total <= 227 * 1024 &&
-         tma_smem_layout<false>(p.f).total <= 227 * 1024;
+  auto ok = [&](int fmt) {
+    return (fmt == 4 && tma_fits<4>(p)) || (fmt == 8 && tma_fits<8>(p));
+  };
+  return ok(p.routed.fmt) && (!p.has_shared || ok(p.shared.fmt));
 }
 
 cudaError_t launch_tma_gate_up(const Plan& p, cudaStream_t st, bool pdl) {

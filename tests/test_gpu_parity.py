@@ -173,7 +173,9 @@ def test_tc_formats_many_rows_per_expert(B, fmt):
 @pytest.mark.parametrize("T,path", [(1, "auto"), (5, "gemv"), (96, "tc")])
 def test_mixed_bank_formats(B, routed, shared, T, path):
     """The shared expert in another encoding than the routed experts: the grouped products
-    run once per bank (the single-kernel and TMA GEMV paths decline such layers)."""
+    run once per bank (the TMA GEMV takes int4/int8 pairs, one launch per bank; a bf16 bank
+    takes the register-streaming GEMV; the single-kernel 1-token layer declines such
+    layers)."""
     cfg = synth.LayerConfig(f"mixed-{routed}-{shared}", T=T, d=384, E=12, k=3, f=256,
                             n_shared=1, fmt=routed, shared_fmt=shared, seed=19)
     L = synth.make_layer(cfg)
@@ -181,11 +183,14 @@ def test_mixed_bank_formats(B, routed, shared, T, path):
     check_layer(B, B.DeviceLayer(L), L, L.x, path)
 
 
-def test_gemv_path_row_invariance(B):
+@pytest.mark.parametrize("routed,shared", [("int4", "int4"), ("int8", "int8"), ("int4", "int8")])
+def test_gemv_path_row_invariance(B, routed, shared):
     """On the GEMV path a token's output bits do not depend on the other tokens of the call
     (up to 32): the first T rows of a 32-token call equal a T-token call bit for bit, and
-    permuting the tokens permutes the outputs bit for bit."""
-    cfg = synth.LayerConfig("ri", T=32, d=512, E=64, k=4, f=256, n_shared=1, fmt="int4", seed=23)
+    permuting the tokens permutes the outputs bit for bit (int8 banks and W8 shared beside
+    W4 routed on the TMA GEMV too)."""
+    cfg = synth.LayerConfig("ri", T=32, d=512, E=64, k=4, f=256, n_shared=1, fmt=routed,
+                            shared_fmt=shared, seed=23)
     L = synth.make_layer(cfg)
     dl = B.DeviceLayer(L)
     x = torch.from_numpy(L.x.view(np.int16)).cuda().view(torch.bfloat16)
@@ -201,6 +206,18 @@ def test_gemv_path_row_invariance(B):
         assert torch.equal(run(x[:T]), o32[:T]), T
     perm = torch.randperm(32, generator=torch.Generator().manual_seed(1)).cuda()
     assert torch.equal(run(x[perm]), o32[perm])
+
+
+@pytest.mark.parametrize("routed,shared,T", [("int8", "int8", 1), ("int8", "int8", 16),
+                                             ("int4", "int8", 1), ("int4", "int8", 32)])
+def test_w8_layers_full_size_gemv(B, routed, shared, T):
+    """W8 edge layers (int8 routed and shared) and a W8 shared expert beside W4 routed
+    experts, at the decode/verify layer size, on the automatic path (the TMA GEMV kernels up
+    to 32 rows): every row against the oracle."""
+    cfg = synth.LayerConfig(f"w8-{routed}-{shared}", T=T, d=2560, E=512, k=10, f=1024,
+                            fmt=routed, shared_fmt=shared, seed=31)
+    L = synth.make_layer(cfg)
+    check_layer(B, B.DeviceLayer(L), L, L.x, "auto", check_stages=False)
 
 
 def test_tc_tiny(B, tiny):
