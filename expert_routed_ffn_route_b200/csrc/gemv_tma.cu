@@ -73,8 +73,11 @@ __host__ __device__ inline TmaSmem tma_smem_layout(int K) {
   return m;
 }
 
-// Tile -> expert and rows. Slots 0..n_active-1 are the active routed experts (ascending
-// ids), slot n_active is the shared expert.
+// Tile -> expert and rows. Tiles [0, n_active * n_rowtiles) are the active routed experts'
+// (ascending ids; all of an expert's rows), then the shared expert's: one tile per (kTok-row
+// token chunk, row tile), chunk-major, so every tile carries at most kTok rows and a CTA's
+// consecutive shared tiles use the same staged rows. (The shared expert's T rows taken
+// whole cost a CTA 3.6x a routed tile at 16 rows, restaging its rows for every chunk.)
 struct TileInfo {
   int slot, e, shared, row_begin, nrows, rowtile;
 };
@@ -82,20 +85,29 @@ struct TileInfo {
 __device__ __forceinline__ TileInfo tile_info(const Plan& p, int ti, int n_rowtiles,
                                               int n_active) {
   TileInfo t;
-  t.slot = ti / n_rowtiles;
-  t.rowtile = ti % n_rowtiles;
-  if (t.slot < n_active) {
+  const int n_rt = n_active * n_rowtiles;
+  if (ti < n_rt) {
+    t.slot = ti / n_rowtiles;
+    t.rowtile = ti % n_rowtiles;
     t.e = p.active[1 + t.slot];
     t.shared = 0;
     t.row_begin = p.offsets[t.e];
     t.nrows = p.offsets[t.e + 1] - t.row_begin;
   } else {
+    const int j = ti - n_rt;
+    t.slot = n_active;
+    t.rowtile = j % n_rowtiles;
     t.e = 0;
     t.shared = 1;
-    t.row_begin = 0;
-    t.nrows = p.T;
+    t.row_begin = (j / n_rowtiles) * kTok;
+    t.nrows = min(kTok, p.T - t.row_begin);
   }
   return t;
+}
+
+// Tiles of the shared expert: one per (token chunk, row tile).
+__host__ __device__ __forceinline__ int shared_tiles(int T, int n_rowtiles) {
+  return ((T + kTok - 1) / kTok) * n_rowtiles;
 }
 
 // Stage the activation rows of token chunk c0 of tile t (x gathered through perm for the
@@ -157,20 +169,14 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p, int pa
 
   const int n_active = p.active[0];
   const int n_rowtiles = N / Sh::ROWS;
-  // Contiguous tile ranges balanced by cost: a routed tile (a few rows) costs 1, a shared-
-  // expert tile (all T rows) costs its kTok-row chunks. A CTA takes the tiles whose cost
-  // interval starts inside its share [c0, c1) of the total (the partition moves no
+  // Contiguous, equal tile ranges over the tiles of this launch (the partition moves no
   // arithmetic: every tile is computed the same way whichever CTA takes it).
   const int n_rt = (part == 2) ? 0 : n_active * n_rowtiles;
-  const int n_st = (p.has_shared && part != 1) ? n_rowtiles : 0;
+  const int n_st = (p.has_shared && part != 1) ? shared_tiles(p.T, n_rowtiles) : 0;
   const int tile0 = (part == 2) ? n_active * n_rowtiles : 0;  // numbering of the full list
-  const int s_cost = (p.T + kTok - 1) / kTok;
-  const long long total_cost = (long long)n_rt + (long long)n_st * s_cost;
-  auto first_tile = [&](long long c) -> int {
-    return c <= n_rt ? (int)c : n_rt + (int)((c - n_rt + s_cost - 1) / s_cost);
-  };
-  const int t_begin = tile0 + first_tile(total_cost * blockIdx.x / gridDim.x);
-  const int t_end = tile0 + first_tile(total_cost * (blockIdx.x + 1) / gridDim.x);
+  const long long n_tiles = (long long)n_rt + n_st;
+  const int t_begin = tile0 + (int)(n_tiles * blockIdx.x / gridDim.x);
+  const int t_end = tile0 + (int)(n_tiles * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == kCons) {
     // ------------------------------------------------------------ producer
@@ -208,14 +214,14 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p, int pa
   const int ctid = threadIdx.x;  // 0 .. 255
   const int rt = warp / Sh::KS, ks = warp % Sh::KS;
   const int grp = lane >> 2, q4 = lane & 3;
-  int staged_slot = -1, staged_c0 = -1;
+  int staged_slot = -1, staged_c0 = -1;  // the staged rows: slot and first grouped row
   int i = 0;
   for (int ti = t_begin; ti < t_end; ++ti, ++i) {
     const int s = i % Sh::NS, u = i / Sh::NS;
     const TileInfo t = tile_info(p, ti, n_rowtiles, n_active);
     // The first token chunk of a new expert is staged before the wait for the tile's
     // weights, so the activation loads overlap the weight copies.
-    const bool pre = (staged_slot != t.slot || staged_c0 != 0);
+    const bool pre = (staged_slot != t.slot || staged_c0 != t.row_begin);
     if (pre) stage_tile_rows<FMT, GATE_UP>(p, t, 0, K, xs, S, xsum, ctid);
     if (ctid == 0) flag[1] = mbar_wait(&full[s], u & 1) ? 1 : 0;
     named_bar_sync(1, 32 * kCons);
@@ -225,19 +231,19 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p, int pa
     }
     if (pre) {
       staged_slot = t.slot;
-      staged_c0 = 0;
+      staged_c0 = t.row_begin;
     }
     const uint8_t* st = smem + (size_t)s * L.stage_bytes;
     const int la = rt * 16 + grp, lb = la + 8;  // rows inside the tile
 
     for (int c0 = 0; c0 < t.nrows; c0 += kTok) {
       const int nr = min(kTok, t.nrows - c0);
-      if (staged_slot != t.slot || staged_c0 != c0) {
+      if (staged_slot != t.slot || staged_c0 != t.row_begin + c0) {
         named_bar_sync(1, 32 * kCons);  // everyone is done with the previous rows
         stage_tile_rows<FMT, GATE_UP>(p, t, c0, K, xs, S, xsum, ctid);
         named_bar_sync(1, 32 * kCons);
         staged_slot = t.slot;
-        staged_c0 = c0;
+        staged_c0 = t.row_begin + c0;
       }
       float acc[NM][4];
 #pragma unroll
@@ -292,7 +298,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) gemv_tma_kernel(Plan p, int pa
           const size_t hrow = (t.shared ? (size_t)p.T * p.k : 0) + t.row_begin + c0 + tok;
           p.h[hrow * p.f + n] = f32_to_bf16_rn(hval);
         } else {
-          float* dst = t.shared ? p.y_shared + (size_t)(c0 + tok) * p.d
+          float* dst = t.shared ? p.y_shared + (size_t)(t.row_begin + c0 + tok) * p.d
                                 : p.y_assign + (size_t)(t.row_begin + c0 + tok) * p.d;
           dst[n] = tot[0];
         }
