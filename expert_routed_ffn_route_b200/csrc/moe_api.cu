@@ -205,10 +205,10 @@ bool scales_aligned16(const Bank& b) {
 // Up to 32 rows (decode and speculative-verify calls) the automatic choice keeps a token's
 // output bits independent of the call: the GEMV kernels and the single-kernel 1-token layer
 // share one arithmetic order (TandemLLM docs, "17 Qwen3.8-Flash-Next", §17.3: decode rows
-// must equal the rows of a verify chain bit for bit). The tensor cores would run 16- and
-// 32-row calls about 15% faster (measured on B200: 291 / 473 against 334 / 555 us) but sum
-// in another order; MOE_PATH_TC asks for them. Kernels after the first of a call use
-// programmatic dependent launch.
+// must equal the rows of a verify chain bit for bit); they are also the faster choice
+// there (measured on B200: 16 / 32 rows 233 / 387 us against 289 / 473 us on the tensor
+// cores, which sum in another order; MOE_PATH_TC asks for them). Kernels after the first of
+// a call use programmatic dependent launch.
 bool use_tc(const Plan& p) {
   if (p.path == MOE_PATH_GEMV || p.path == MOE_PATH_FUSED) return false;
   if (p.path == MOE_PATH_TC) return true;

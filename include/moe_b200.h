@@ -96,8 +96,7 @@ typedef enum { MOE_W_BF16 = 16, MOE_W_INT8 = 8, MOE_W_INT4 = 4, MOE_W_NVFP4 = 41
  * row-invariant: a token's output (and its routing) is the same bits whether it is called
  * alone or among up to 32 rows, in any position (the single-kernel layer and the GEMV
  * kernels share one arithmetic order; TandemLLM docs, "17 Qwen3.8-Flash-Next", §17.3).
- * TC asks for the tensor cores at any T (faster for 16..32 rows, not row-invariant with the
- * 1-token layer). FUSED asks for the single-kernel layer and returns MOE_ERR_UNSUPPORTED
+ * TC asks for the tensor cores at any T (not row-invariant with the 1-token layer). FUSED asks for the single-kernel layer and returns MOE_ERR_UNSUPPORTED
  * from moe_layer_forward when the call does not fit it; the stage entry points (moe_route ...
  * moe_combine) treat FUSED like GEMV. NVFP4 layers run on the FP4 tensor cores for every T. */
 typedef enum { MOE_PATH_AUTO = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC = 2, MOE_PATH_FUSED = 3 } moe_path;
