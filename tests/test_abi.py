@@ -123,6 +123,25 @@ def test_nvfp4_helpers_validate_on_host(lib):
     assert q(fake + 8, 4, 64, fake, fake, fake, None) == -1        # alignment
 
 
+def test_launch_counts_follow_the_automatic_path(lib):
+    """Host-side path choice (no GPU needed above one row): up to 32 rows the fused routing
+    kernel, the two GEMV kernels and the combine (4 launches); from 33 rows router, top-k, the
+    plan, the tensor-core prep, gate/up and down, and the combine; a W8 shared expert beside
+    W4 routed experts runs each GEMM once per bank; NVFP4 routed experts add the activation
+    quantisers and the shared expert's own GEMMs."""
+    for T in (2, 16, 32):
+        assert lib.moe_launches_per_call(ctypes.byref(_desc(T=T))) == 4, T
+    assert lib.moe_launches_per_call(ctypes.byref(_desc(T=33))) == 7  # 330 assignments: one plan kernel
+    assert lib.moe_launches_per_call(ctypes.byref(_desc(T=512))) == 9  # the plan in 3 kernels
+    d = _desc(T=16)
+    d.shared.fmt = 8
+    assert lib.moe_launches_per_call(ctypes.byref(d)) == 6
+    d = _desc(T=16)
+    d.path = binding.PATH_CODE["tc"]
+    assert lib.moe_launches_per_call(ctypes.byref(d)) == 5
+    assert lib.moe_launches_per_call(ctypes.byref(_nvfp4_desc(T=16))) == 1 + 5 + 2 + 1
+
+
 def test_workspace_size_grows_with_T(lib):
     a = lib.moe_workspace_size(ctypes.byref(_desc(T=1)))
     b = lib.moe_workspace_size(ctypes.byref(_desc(T=4096)))

@@ -137,6 +137,29 @@ def test_rows_are_independent():
         np.testing.assert_allclose(one[0], full[t], rtol=1e-12, atol=1e-16)  # BLAS order aside
 
 
+def test_token_subset_equals_the_full_call():
+    """The ``tokens`` option computes the listed rows only (routing and the plan stay those of
+    the whole call): each listed row equals the full call's row, in the order listed (up to the
+    fp64 matrix routine's summation order over a different number of rows)."""
+    cfg, L, routed, shared = _layer(T=6)
+    full = N.layer_forward_nvfp4(L.x, L.router_w, L.router_bias, routed, shared, cfg.k)
+    sub = N.layer_forward_nvfp4(L.x, L.router_w, L.router_bias, routed, shared, cfg.k,
+                                tokens=[4, 1, 5])
+    np.testing.assert_allclose(sub["out"], full["out"][[4, 1, 5]], rtol=1e-12, atol=1e-16)  # BLAS order aside
+    assert np.array_equal(sub["idx"], full["idx"]) and np.array_equal(sub["perm"], full["perm"])
+
+
+def test_generator_e2m1_rounding_matches_the_oracle():
+    """The generator's vectorised E2M1 rounding (which fixes the stored weight codes) takes
+    the oracle's decisions: nearest, ties to the even code, saturation at 6, the sign bit."""
+    rng = np.random.default_rng(13)
+    grid = N.e2m1_value(np.arange(8))
+    mids = (grid[1:] + grid[:-1]) / 2
+    v = np.concatenate([rng.uniform(-8, 8, 20000), mids, -mids, grid, -grid,
+                        [6.5, -7.0, 0.0, -0.0, 1e-9, -1e-9]]).astype(np.float32)
+    assert np.array_equal(synth.e2m1_codes(v).astype(np.int64), N.round_e2m1(v))
+
+
 def _unquantised_error(layer_fn):
     cfg, L, routed, shared = _layer(T=8, E=6, k=2, seed=11)
     w4a4 = layer_fn(L.x, L.router_w, L.router_bias, routed, shared, cfg.k)["out"]
