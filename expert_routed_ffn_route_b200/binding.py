@@ -103,6 +103,16 @@ def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
+def bank_struct(b) -> MoeBank:
+    """A bank dict (fmt, group, n_exp and device tensors w_*, s_*, g_*) -> moe_bank."""
+    if b is None:
+        return MoeBank(16, 128, 0, 0, None, None, None, None, None, None, None, None, None)
+    return MoeBank(FMT_CODE[b["fmt"]], b["group"], b["n_exp"], 0,
+                   _ptr(b["w_gate"]), _ptr(b["w_up"]), _ptr(b["w_down"]),
+                   _ptr(b.get("s_gate")), _ptr(b.get("s_up")), _ptr(b.get("s_down")),
+                   _ptr(b.get("g_gate")), _ptr(b.get("g_up")), _ptr(b.get("g_down")))
+
+
 class DeviceLayer:
     """Device-resident inputs of one layer that do not depend on the tokens:
     router weights, optional router bias, routed and shared expert banks."""
@@ -152,12 +162,7 @@ class DeviceLayer:
         return self
 
     def _bank(self, b) -> MoeBank:
-        if b is None:
-            return MoeBank(16, 128, 0, 0, None, None, None, None, None, None, None, None, None)
-        return MoeBank(FMT_CODE[b["fmt"]], b["group"], b["n_exp"], 0,
-                       _ptr(b["w_gate"]), _ptr(b["w_up"]), _ptr(b["w_down"]),
-                       _ptr(b.get("s_gate")), _ptr(b.get("s_up")), _ptr(b.get("s_down")),
-                       _ptr(b.get("g_gate")), _ptr(b.get("g_up")), _ptr(b.get("g_down")))
+        return bank_struct(b)
 
     def descriptor(self, T: int, path: str | None = None) -> MoeLayer:
         return MoeLayer(T, self.d, self.f, self.E, self.k,
