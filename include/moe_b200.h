@@ -80,7 +80,7 @@ typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = -1, /* a pointer, size, alignment or shape is not accepted   */
-  MOE_ERR_UNSUPPORTED = -2, /* a valid request this build does not implement         */
+  MOE_ERR_UNSUPPORTED = -2, /* a valid request the library does not implement       */
   MOE_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch or attribute)       */
   MOE_ERR_TIMEOUT = -4,     /* a bounded device-side wait gave up (device status)     */
   MOE_ERR_WORKSPACE = -5,   /* workspace NULL, misaligned or smaller than required    */

@@ -2,8 +2,8 @@
 ranks over gloo: the exchange plumbing, the owner ranges and the fixed-order combine.
 
 Each rank's arithmetic is given by the fp64 oracle here (``OracleOps``); on GPUs the same
-layer runs the library's stage entry points (``LibraryOps``), which one GPU a call does not let
-this suite run as several ranks. The expert-parallel result on every rank equals the
+layer runs the library's stage entry points (``LibraryOps``; tests/test_gpu_expert_parallel.py
+runs two such ranks sharing one device). The expert-parallel result on every rank equals the
 single-process oracle layer on that rank's tokens (up to the fp64 matrix routine's order), for
 2 and 4 ranks, with uneven token counts per rank, and is the same bits when repeated."""
 import os
