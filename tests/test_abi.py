@@ -168,3 +168,23 @@ def test_launch_count_of_mixed_bank_formats(lib, path, single):
     assert lib.moe_launches_per_call(ctypes.byref(d)) == single
     d.shared.fmt = 8
     assert lib.moe_launches_per_call(ctypes.byref(d)) == single + 2
+
+
+def test_header_is_plain_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as C99 (no C++ types in the signatures),
+    and the struct layout the binding declares matches the compiler's."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "moe_b200.h"\n'
+                   'int main(void) { printf("%zu %zu %zu %zu\\n", sizeof(moe_bank), sizeof(moe_layer),'
+                   ' offsetof(moe_layer, routed), offsetof(moe_bank, g_gate)); return 0; }\n')
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    sizes = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                            check=True).stdout.split()]
+    assert sizes == [ctypes.sizeof(binding.MoeBank), ctypes.sizeof(binding.MoeLayer),
+                     binding.MoeLayer.routed.offset, binding.MoeBank.g_gate.offset]
